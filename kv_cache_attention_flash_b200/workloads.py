@@ -1,0 +1,345 @@
+"""Seeded synthetic workloads for the Flash-dLLM per-layer step.
+
+This module only draws inputs. It holds none of the step's arithmetic: no
+projection, no rotary embedding, no attention, no rounding of results. Both
+the CUDA path and the CPU oracle consume what it produces, so it is the one
+piece of code they share.
+
+The five workloads mirror the settings the Flash-dLLM pages describe for
+LLaDA-1.5 serving ("Flash-dLLM: I/O-Aware KV Caching and Parallel Decoding
+for Fast, Memory-Efficient Diffusion LLMs", ai4snews summary of the full
+text, paragraphs 1-4): a single layer at LLaDA-8B shape, a batch of 32
+sequences whose lengths and stages diverge, the Flash-Verify two-view block,
+and a 32-layer stack. No public benchmark data is used; every tensor is
+drawn from a seeded generator.
+
+Recipe (all seeds fixed by the caller):
+  * metadata (lengths, positions, stages, page permutation) from
+    ``numpy.random.default_rng(seed)``;
+  * x ~ N(0, 1), Wqkv ~ N(0, 0.02^2), drawn as float32 by a seeded
+    ``torch.Generator`` and cast to the workload dtype (bf16 casts round to
+    nearest even);
+  * the pre-existing cache holds N(0, 1.28^2) values in the visible slots
+    (1.28^2 ~= H * 0.02^2, the second moment of a projected key), a NaN bit
+    pattern in every slot this step writes and in every page tail past the
+    sequence's last slot, and random bits in spare pages.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, List, Optional
+
+import numpy as np
+import torch
+
+BF16_NAN_BITS = 0x7FC1      # a quiet NaN that no arithmetic produces by itself
+F32_NAN_BITS = 0x7FC00011
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerShape:
+    dtype: str            # "bf16" or "f32": x, Wqkv and the cache pools
+    hidden: int
+    n_heads: int
+    head_dim: int
+    page_size: int
+    rope_theta: float
+    n_layers: int = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class WorkloadSpec:
+    name: str
+    shape: LayerShape
+    batch: int
+    kind: str                     # "window", "divergent", "two_view"
+    ctx_len: int = 0              # fixed visible context (window / two_view)
+    prompt_len: int = 0           # window start is drawn after the prompt
+    ctx_min: int = 0              # divergent: L_b ~ U[ctx_min, ctx_max]
+    ctx_max: int = 0
+    window: int = 32
+    tracked: int = 32             # tracked rows per update-stage sequence
+    track_k: int = 32             # k of the next step's top-k selection
+    view_rows: int = 32           # two_view: rows per view
+    spare_pages: int = 4
+
+
+LLADA8B = LayerShape("bf16", 4096, 32, 128, 64, 500000.0)
+
+WORKLOADS: Dict[str, WorkloadSpec] = {
+    # Tiny single layer, fp32; 64 prompt + 64 generated slots, 16-slot pages.
+    "tiny_f32": WorkloadSpec("tiny_f32", LayerShape("f32", 256, 4, 64, 16, 10000.0),
+                             batch=1, kind="window", ctx_len=128, prompt_len=64,
+                             window=8, tracked=8, track_k=8, spare_pages=3),
+    # LLaDA-8B-shaped layer, batch 1, 256 prompt + 512 generated slots.
+    "llada8b_b1": WorkloadSpec("llada8b_b1", LLADA8B, batch=1, kind="window",
+                               ctx_len=768, prompt_len=256, window=32, tracked=32, track_k=32),
+    # Batch 32, L_b ~ U[256, 1024], half caching stage (window only), half
+    # update stage (window + 32 tracked), pages permuted in the pool.
+    "b32_divergent": WorkloadSpec("b32_divergent", LLADA8B, batch=32, kind="divergent",
+                                  ctx_min=256, ctx_max=1024, window=32, tracked=32, track_k=32,
+                                  spare_pages=8),
+    # Flash-Verify two views: 32 draft + 32 mask rows at the same positions.
+    "two_view_b8": WorkloadSpec("two_view_b8", LLADA8B, batch=8, kind="two_view",
+                                ctx_len=1024, view_rows=32, track_k=32),
+    # 32 stacked layers, batch 4, 8192 context slots, 32 window + 64 tracked.
+    "stacked32_b4": WorkloadSpec("stacked32_b4", dataclasses.replace(LLADA8B, n_layers=32),
+                                 batch=4, kind="window", ctx_len=8192, prompt_len=0,
+                                 window=32, tracked=64, track_k=64),
+}
+
+# Small variants of the same structure (same code paths, oracle-sized).
+SMALL_WORKLOADS: Dict[str, WorkloadSpec] = {
+    "small_bf16_divergent": WorkloadSpec(
+        "small_bf16_divergent", LayerShape("bf16", 512, 4, 128, 64, 500000.0),
+        batch=6, kind="divergent", ctx_min=70, ctx_max=400, window=32, tracked=32,
+        track_k=16, spare_pages=3),
+    "small_bf16_two_view": WorkloadSpec(
+        "small_bf16_two_view", LayerShape("bf16", 512, 4, 128, 64, 10000.0),
+        batch=3, kind="two_view", ctx_len=200, view_rows=24, track_k=8, spare_pages=2),
+    "small_f32_divergent": WorkloadSpec(
+        "small_f32_divergent", LayerShape("f32", 128, 2, 64, 16, 10000.0),
+        batch=4, kind="divergent", ctx_min=20, ctx_max=90, window=8, tracked=8,
+        track_k=6, spare_pages=2),
+}
+
+
+def get_spec(name: str) -> WorkloadSpec:
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    return SMALL_WORKLOADS[name]
+
+
+@dataclasses.dataclass
+class StepMeta:
+    """Host-side description of one step (all arrays numpy)."""
+    batch: int
+    cu_rows: np.ndarray       # int32 [B+1]
+    seq_lens: np.ndarray      # int32 [B]  visible context slots L_b
+    positions: np.ndarray     # int32 [R]
+    slots: np.ndarray         # int32 [R]
+    view: np.ndarray          # int8  [R]  0 plain, 1 draft, 2 mask
+    block_table: np.ndarray   # int32 [B, max_blocks]
+    num_pages: int
+    max_position: int         # exclusive bound on positions (RoPE table size)
+    exclude_cu: np.ndarray    # int32 [B+1] exclusion list offsets (the window slots)
+    exclude_slots: np.ndarray  # int32 [E]
+    track_k: int
+    stage: np.ndarray         # int8 [B] 0 caching, 1 update, 2 verify
+
+    @property
+    def total_rows(self) -> int:
+        return int(self.cu_rows[-1])
+
+    @property
+    def max_blocks(self) -> int:
+        return int(self.block_table.shape[1])
+
+
+def _window_and_tracked(rng, L, window, tracked, lo):
+    lo = max(0, min(lo, L - window))
+    start = int(rng.integers(lo, L - window + 1))
+    win = np.arange(start, start + window, dtype=np.int64)
+    rest = np.setdiff1d(np.arange(L, dtype=np.int64), win)
+    trk = np.sort(rng.choice(rest, size=tracked, replace=False)) if tracked else np.zeros(0, np.int64)
+    return win, trk
+
+
+def make_meta(spec: WorkloadSpec, seed: int = 0) -> StepMeta:
+    rng = np.random.default_rng(seed)
+    B = spec.batch
+    ps = spec.shape.page_size
+    rows_pos: List[np.ndarray] = []
+    rows_slot: List[np.ndarray] = []
+    rows_view: List[np.ndarray] = []
+    seq_lens = np.zeros(B, np.int32)
+    need_slots = np.zeros(B, np.int64)
+    excl: List[np.ndarray] = []
+    stage = np.zeros(B, np.int8)
+    if spec.kind == "divergent":
+        stage[:] = 0
+        upd = rng.permutation(B)[: B // 2]
+        stage[upd] = 1
+    for b in range(B):
+        if spec.kind == "two_view":
+            L = spec.ctx_len
+            n = spec.view_rows
+            pos = np.arange(L, L + n, dtype=np.int64)
+            # draft rows write their own positions, mask rows write scratch
+            # slots right after them; both lie past the visible context.
+            p = np.concatenate([pos, pos])
+            s = np.concatenate([pos, pos + n])
+            v = np.concatenate([np.full(n, 1), np.full(n, 2)])
+            seq_lens[b] = L
+            need_slots[b] = L + 2 * n
+            stage[b] = 2
+            excl.append(np.zeros(0, np.int64))
+        else:
+            if spec.kind == "divergent":
+                L = int(rng.integers(spec.ctx_min, spec.ctx_max + 1))
+                lo = L // 4
+                n_trk = spec.tracked if stage[b] == 1 else 0
+            else:
+                L = spec.ctx_len
+                lo = spec.prompt_len if spec.prompt_len else L // 4
+                n_trk = spec.tracked
+                stage[b] = 1
+            win, trk = _window_and_tracked(rng, L, spec.window, n_trk, lo)
+            p = np.concatenate([win, trk])
+            s = p.copy()
+            v = np.zeros(len(p), np.int64)
+            seq_lens[b] = L
+            need_slots[b] = L
+            excl.append(win)
+        rows_pos.append(p)
+        rows_slot.append(s)
+        rows_view.append(v)
+    cu = np.zeros(B + 1, np.int32)
+    cu[1:] = np.cumsum([len(p) for p in rows_pos])
+    blocks_per = [(int(n) + ps - 1) // ps for n in need_slots]
+    max_blocks = max(blocks_per)
+    num_pages = int(sum(blocks_per)) + spec.spare_pages
+    perm = rng.permutation(num_pages).astype(np.int32)
+    bt = np.full((B, max_blocks), -1, np.int32)
+    k = 0
+    for b in range(B):
+        for i in range(blocks_per[b]):
+            bt[b, i] = perm[k]
+            k += 1
+    positions = np.concatenate(rows_pos).astype(np.int32)
+    max_pos = int(positions.max()) + 1
+    exclude_cu = np.zeros(B + 1, np.int32)
+    exclude_cu[1:] = np.cumsum([len(e) for e in excl])
+    return StepMeta(batch=B, cu_rows=cu, seq_lens=seq_lens, positions=positions,
+                    slots=np.concatenate(rows_slot).astype(np.int32),
+                    view=np.concatenate(rows_view).astype(np.int8), block_table=bt,
+                    num_pages=num_pages, max_position=max_pos,
+                    exclude_cu=exclude_cu,
+                    exclude_slots=(np.concatenate(excl) if excl else np.zeros(0)).astype(np.int32),
+                    track_k=spec.track_k, stage=stage)
+
+
+def torch_dtype(shape: LayerShape) -> torch.dtype:
+    return torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def make_x(spec: WorkloadSpec, meta: StepMeta, seed: int, layer: int = 0,
+           device="cpu") -> torch.Tensor:
+    """x [R, H]: N(0,1). In a two-view step every mask-view row carries the
+    same vector (the [MASK] embedding); draft rows are independent."""
+    H = spec.shape.hidden
+    g = _gen(seed * 1000003 + 17 + layer * 7919, device)
+    x = torch.randn(meta.total_rows, H, generator=g, device=device, dtype=torch.float32)
+    if spec.kind == "two_view":
+        m = torch.randn(1, H, generator=g, device=device, dtype=torch.float32)
+        mask_rows = torch.from_numpy(np.nonzero(meta.view == 2)[0]).to(device)
+        x[mask_rows] = m
+    return x.to(torch_dtype(spec.shape))
+
+
+def make_w(spec: WorkloadSpec, seed: int, layer: int = 0, device="cpu") -> torch.Tensor:
+    """Wqkv [H, 3H] row-major, N(0, 0.02^2); columns are [Q | K | V], each
+    block head-major (head h at columns h*D .. h*D+D-1)."""
+    H = spec.shape.hidden
+    g = _gen(seed * 1000003 + 29 + layer * 104729, device)
+    w = torch.randn(H, 3 * H, generator=g, device=device, dtype=torch.float32) * 0.02
+    return w.to(torch_dtype(spec.shape))
+
+
+def make_pools(spec: WorkloadSpec, meta: StepMeta, seed: int, device="cpu",
+               n_layers: Optional[int] = None):
+    """K and V pools [n_layers, num_pages, n_heads, page_size, head_dim].
+
+    Visible slots hold N(0, 1.28^2); every slot the step writes and every page
+    tail past the sequence's last visible/written slot holds a NaN pattern;
+    spare pages hold random bits."""
+    sh = spec.shape
+    nl = sh.n_layers if n_layers is None else n_layers
+    shape = (nl, meta.num_pages, sh.n_heads, sh.page_size, sh.head_dim)
+    g = _gen(seed * 1000003 + 41, device)
+    dt = torch_dtype(sh)
+    nan_bits = BF16_NAN_BITS if sh.dtype == "bf16" else F32_NAN_BITS
+    int_dt = torch.int16 if sh.dtype == "bf16" else torch.int32
+    pools = []
+    for _ in range(2):
+        # start from random bits everywhere (spare pages keep them)
+        if sh.dtype == "bf16":
+            bits = torch.randint(-32768, 32767, shape, generator=g, device=device, dtype=torch.int16)
+        else:
+            bits = torch.randint(-2**31, 2**31 - 1, shape, generator=g, device=device, dtype=torch.int32)
+        pool = bits.view(dt)
+        ps = sh.page_size
+        for b in range(meta.batch):
+            L = int(meta.seq_lens[b])
+            r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
+            top = max([L] + [int(s) + 1 for s in meta.slots[r0:r1]])
+            nblk = (top + ps - 1) // ps
+            for i in range(nblk):
+                pg = int(meta.block_table[b, i])
+                lo = i * ps
+                n_vis = max(0, min(ps, L - lo))
+                if n_vis:
+                    vals = torch.randn((nl, sh.n_heads, n_vis, sh.head_dim), generator=g,
+                                       device=device, dtype=torch.float32) * 1.28
+                    pool[:, pg, :, :n_vis, :] = vals.to(dt)
+                if n_vis < ps:
+                    pool.view(int_dt)[:, pg, :, n_vis:, :] = nan_bits if sh.dtype == "f32" else _i16(nan_bits)
+            for s in meta.slots[r0:r1]:
+                pg = int(meta.block_table[b, int(s) // ps])
+                pool.view(int_dt)[:, pg, :, int(s) % ps, :] = nan_bits if sh.dtype == "f32" else _i16(nan_bits)
+        pools.append(pool)
+    return pools[0], pools[1]
+
+
+def _i16(u: int) -> int:
+    return u - 65536 if u >= 32768 else u
+
+
+def bits_np(t: torch.Tensor) -> np.ndarray:
+    """Raw bits of a bf16/f32 tensor as uint16/uint32 numpy (host copy)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy().view(np.uint32)
+    raise TypeError(t.dtype)
+
+
+def algorithmic_bytes_flops(spec: WorkloadSpec, meta: StepMeta, with_mass: bool = True):
+    """Byte and FLOP model of one layer step (per layer).
+
+    bytes = Wqkv + x + cache reads of visible non-fresh slots + cache writes
+            + out (fp32) + attn_mass (fp32);
+    flops = 2*R*H*3H (projection) + 4*D*n_h*sum_r |K(r)| (QK^T and PV).
+    The second key pass, padding rows and RoPE/softmax arithmetic are not
+    counted."""
+    sh = spec.shape
+    s = 2 if sh.dtype == "bf16" else 4
+    H = sh.hidden
+    R = meta.total_rows
+    byt = H * 3 * H * s + R * H * s + R * 2 * H * s + R * H * 4
+    fl = 2 * R * H * 3 * H
+    keys = 0
+    for b in range(meta.batch):
+        L = int(meta.seq_lens[b])
+        r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
+        sl = meta.slots[r0:r1]
+        vw = meta.view[r0:r1]
+        ps_ = meta.positions[r0:r1]
+        fresh_vis = int(np.sum((sl < L) & (vw == 0)))
+        byt += (L - fresh_vis) * 2 * H * s
+        if with_mass:
+            byt += 4 * L
+        for i in range(r1 - r0):
+            k = L
+            if vw[i] != 0:
+                k += int(np.sum((vw == vw[i]) & (ps_ <= ps_[i])))
+            keys += k
+    fl += 4 * sh.head_dim * sh.n_heads * keys
+    return byt, fl
