@@ -1,0 +1,202 @@
+/*
+ * fdllm.h - C ABI of the Flash-dLLM per-layer hot path on NVIDIA B200 (sm_100a).
+ *
+ * One layer step of masked-diffusion decoding with Flash-dLLM KV caching:
+ *   (a) Flash-Cache: the selected rows' hidden states go through the QKV
+ *       projection, RoPE is applied, and K/V are written from on-chip memory
+ *       straight into a paged KV cache; Q never leaves the SM.
+ *   (b) scheduled attention: each sequence's query rows attend over that
+ *       sequence's pages through its block table, so one launch covers a
+ *       batch whose sequences differ in length and in stage; the Flash-Verify
+ *       two-view mask is applied inside the same kernel, and each key's
+ *       accumulated attention mass is emitted for the next step's top-k
+ *       tracking set.
+ *
+ * Sources (cited by page title and paragraph):
+ *   [FD] "Flash-dLLM: I/O-Aware KV Caching and Parallel Decoding for Fast,
+ *        Memory-Efficient Diffusion LLMs" (ai4snews summary of the full text).
+ *        Paragraph 1: Flash-Cache fuses QKV projection, RoPE and the cache
+ *        write; scheduled Flash Attention aligns query blocks with their KV
+ *        blocks through a block table across caching and update stages.
+ *        Paragraph 2: each step's queries are a sliding unmasking window plus
+ *        a fixed tracking budget of most-attended tokens.
+ *        Paragraph 3: Flash-Verify places a draft view and a mask view at the
+ *        same positions, sharing positional embeddings, isolated from each
+ *        other by a causal mask inside the fused kernel.
+ *   [AB] "Flash-dLLM: IO-Aware KV Caching and Parallel Decoding for Fast,
+ *        Memory-Efficient Diffusion LLMs" (arXiv abstract page), Abstract:
+ *        GPU memory I/O is the dominant bottleneck; an I/O-aware fused
+ *        KV-cache kernel reduces redundant memory movement.
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented DEVICE are CUDA device pointers owned by the
+ *     caller and borrowed for the duration of the call (and of the work it
+ *     enqueues). Pointers documented HOST are read before the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued asynchronously; nothing synchronises except
+ *     fdllm_check, fdllm_cache_create and steps run with validate = 1.
+ *   - Host-detectable errors return a status and enqueue nothing.
+ *     fdllm_last_error() returns a message for the calling thread.
+ *   - Device-detected errors (a page id outside the pool, a slot past the
+ *     block table, a position outside the RoPE table) skip the offending
+ *     row, never trap, and are reported by the next fdllm_check as
+ *     FDLLM_ERR_DEVICE_BOUNDS.
+ *   - The library is single-GPU: every pointer must live on the device that
+ *     was current at fdllm_cache_create.
+ */
+#ifndef FDLLM_H
+#define FDLLM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FDLLM_API __attribute__((visibility("default")))
+#else
+#define FDLLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FDLLM_OK = 0,
+  FDLLM_ERR_INVALID_ARG = 1,   /* bad pointer, size or shape (host check) */
+  FDLLM_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels cover */
+  FDLLM_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  FDLLM_ERR_DEVICE_BOUNDS = 4, /* a kernel found out-of-range metadata */
+  FDLLM_ERR_TIMEOUT = 5        /* a bounded in-kernel wait gave up */
+} fdllm_status;
+
+typedef enum { FDLLM_BF16 = 0, FDLLM_F32 = 1 } fdllm_dtype;
+
+/* Shape of the paged KV cache and of the layer it serves.
+ *   n_layers, n_heads, head_dim, page_size, num_pages: pool geometry.
+ *   hidden = n_heads * head_dim (no grouped-query attention).
+ *   max_position: RoPE positions must lie in [0, max_position).
+ *   rope_theta: RoPE base (rotate-half pairing (i, i + head_dim/2), angle
+ *     p * rope_theta^(-2i/head_dim); [FD] paragraph 1 fuses RoPE with the
+ *     projection, the form is the LLaMA-family one).
+ *   max_batch, max_slots_per_seq: bounds used to size the library's
+ *     attention-mass workspace (n_heads * max_batch * max_slots_per_seq
+ *     floats). A step with batch > max_batch or
+ *     max_blocks_per_seq * page_size > max_slots_per_seq is rejected.
+ *   dtype: FDLLM_BF16 (x, Wqkv, pools in bf16; fp32 accumulation) or
+ *     FDLLM_F32 (everything fp32). */
+typedef struct {
+  int32_t n_layers;
+  int32_t n_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t num_pages;
+  int32_t max_position;
+  int32_t max_batch;
+  int32_t max_slots_per_seq;
+  float rope_theta;
+  int32_t dtype; /* fdllm_dtype */
+} fdllm_cache_config;
+
+typedef struct fdllm_cache fdllm_cache; /* opaque */
+
+/* Per-step description.
+ *   batch: sequences in the step (1 .. 256).
+ *   total_rows: R = cu_rows[batch].
+ *   max_blocks_per_seq: row length of block_table.
+ *   cu_rows: HOST int32 [batch+1], row offsets of each sequence into x/out;
+ *     a sequence holds at most 128 rows.
+ *   seq_lens: HOST int32 [batch], L_b = visible context slots of sequence b
+ *     (slots [0, L_b) through its block table).
+ *   slots: DEVICE int32 [total_rows], cache slot each row writes; NULL means
+ *     slot = position.
+ *   validate: 1 = copy the device metadata to the host and check it before
+ *     launching (slow; for tests). Duplicate slots within a sequence and
+ *     view rows writing inside [0, L_b) are only detected this way. */
+typedef struct {
+  int32_t batch;
+  int32_t total_rows;
+  int32_t max_blocks_per_seq;
+  const int32_t* cu_rows;
+  const int32_t* seq_lens;
+  const int32_t* slots;
+  int32_t validate;
+} fdllm_step;
+
+/* Creates a handle over caller-owned pools.
+ *   k_pool, v_pool: DEVICE [n_layers][num_pages][n_heads][page_size][head_dim]
+ *     of cfg->dtype, 16-byte aligned. Not modified here.
+ * Allocates the RoPE cos/sin tables (computed on the host in double,
+ * stored fp32), the mass workspace and a device error word, and
+ * synchronises `stream` once. */
+FDLLM_API fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, void* v_pool,
+                                void* stream, fdllm_cache** out);
+
+/* Frees what fdllm_cache_create allocated (not the pools). NULL is a no-op. */
+FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
+
+/* One Flash-Cache + scheduled-attention layer step ([FD] paragraphs 1-3).
+ *   layer: which layer's slice of the pools to write and read.
+ *   x: DEVICE [total_rows][hidden] of the cache dtype, the selected rows'
+ *     hidden states (window rows, tracked rows, or the two views).
+ *   wqkv: DEVICE [hidden][3*hidden] row-major; columns are [Q | K | V], each
+ *     block head-major (head h at columns h*head_dim .. +head_dim-1).
+ *   positions: DEVICE int32 [total_rows], RoPE positions.
+ *   block_table: DEVICE int32 [batch][max_blocks_per_seq], physical page of
+ *     each logical page (slot s of sequence b lives in page
+ *     block_table[b][s / page_size] at offset s % page_size).
+ *   view_mask: DEVICE int8 [total_rows]: 0 plain row, 1 draft view, 2 mask
+ *     view; NULL = all plain. Every row sees the slots [0, L_b) as they
+ *     stand after this step's writes. A view row also sees the slots that
+ *     rows of its own view write in this step at positions <= its own; the
+ *     two views never see each other's fresh slots. View rows must write
+ *     slots >= L_b.
+ *   out: DEVICE fp32 [total_rows][hidden], softmax(q k^T / sqrt(head_dim)) v
+ *     per head, heads concatenated.
+ *   attn_mass: DEVICE fp32 [batch][max_blocks_per_seq * page_size] or NULL.
+ *     attn_mass[b][s] = (1 / (R_b * n_heads)) * sum over heads and over the
+ *     rows of b of the attention probability on slot s; zero for slots
+ *     nobody attends. Each sequence with rows sums to 1 ([FD] paragraph 2:
+ *     the statistic behind the most-attended tracking set).
+ * Writes: out, attn_mass, and for every row the k/v of every head into its
+ * slot; no other cache byte changes. Within one step no sequence may read a
+ * slot another sequence writes. */
+FDLLM_API fdllm_status fdllm_layer_step(fdllm_cache* cache, int32_t layer, const fdllm_step* step,
+                              const void* x, const void* wqkv, const int32_t* positions,
+                              const int32_t* block_table, const int8_t* view_mask, float* out,
+                              float* attn_mass, void* stream);
+
+/* Next step's tracked set ([FD] paragraph 2: a fixed budget of the most
+ * attended tokens).
+ *   attn_mass: DEVICE fp32 [batch][row_stride], non-negative.
+ *   seq_lens: DEVICE int32 [batch]; candidates are slots [0, L_b), L_b <= row_stride,
+ *     L_b <= 65536.
+ *   k: budget, 1 .. 1024.
+ *   exclude_cu: DEVICE int32 [batch+1] or NULL; exclude_slots: DEVICE int32,
+ *     slots removed from sequence b's candidates are
+ *     exclude_slots[exclude_cu[b] .. exclude_cu[b+1]) (out-of-range entries
+ *     are ignored).
+ *   tracked: DEVICE int32 [batch][k]: the k candidates of largest mass in
+ *     descending order, ties to the lower slot, padded with -1. */
+FDLLM_API fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_t* seq_lens, int32_t batch,
+                                  int32_t row_stride, int32_t k, const int32_t* exclude_cu,
+                                  const int32_t* exclude_slots, int32_t* tracked, void* stream);
+
+/* Synchronises `stream`, reads and clears the handle's device error word.
+ * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
+ * FDLLM_ERR_CUDA. */
+FDLLM_API fdllm_status fdllm_check(fdllm_cache* cache, void* stream);
+
+/* Static description of a status code. */
+FDLLM_API const char* fdllm_status_string(fdllm_status status);
+
+/* Message for the last failing call on this thread ("" if none). */
+FDLLM_API const char* fdllm_last_error(void);
+
+/* Number of kernel launches the last successful fdllm_layer_step or
+ * fdllm_select_tracked call on this thread enqueued. */
+FDLLM_API int32_t fdllm_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FDLLM_H */

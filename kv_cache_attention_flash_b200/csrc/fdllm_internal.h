@@ -1,0 +1,73 @@
+// Internal declarations shared by the host API and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fdllm {
+
+constexpr int kMaxBatch = 256;        // sequences per step
+constexpr int kMaxGroups = 256;       // 128-row groups per step
+constexpr int kGroupRows = 128;       // rows per group (the MMA's M)
+constexpr int kMaxSeqRows = 128;      // rows per sequence
+
+// Device error word layout (int32[4]).
+enum DevErr : int {
+  kDevOk = 0,
+  kDevBadPage = 1,      // block table entry outside [0, num_pages)
+  kDevBadSlot = 2,      // slot < 0 or past max_blocks_per_seq * page_size
+  kDevBadPosition = 3,  // position outside [0, max_position)
+  kDevTimeout = 4,      // a bounded wait gave up
+};
+
+// Step plan: built on the host from cu_rows/seq_lens, passed by value.
+struct StepPlan {
+  int batch;
+  int total_rows;
+  int n_groups;
+  int max_blocks;        // block table row length
+  int row_stride;        // max_blocks * page_size (mass row length)
+  int layer;
+  int group_row0[kMaxGroups + 1];  // group g: rows [group_row0[g], group_row0[g+1])
+  int group_seq0[kMaxGroups + 1];  // group g: sequences [group_seq0[g], group_seq0[g+1])
+  int cu_rows[kMaxBatch + 1];
+  int seq_lens[kMaxBatch];
+};
+
+// Per-call device pointers and pool geometry.
+struct StepArgs {
+  const void* x;
+  const void* wqkv;
+  const int32_t* positions;
+  const int32_t* slots;          // may be null: slot = position
+  const int32_t* block_table;
+  const int8_t* view;            // may be null: all plain
+  float* out;
+  float* mass_part;              // [n_heads][batch][row_stride] or null
+  void* k_pool;
+  void* v_pool;
+  const float* rope_cos;         // [max_position][head_dim/2]
+  const float* rope_sin;
+  int* err;                      // device error word
+  int hidden;
+  int n_heads;
+  int head_dim;
+  int page_size;
+  int num_pages;
+  int max_position;
+};
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* tmap_x,
+                             const void* tmap_w, cudaStream_t stream);
+cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream);
+cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
+                               cudaStream_t stream);
+cudaError_t launch_select_tracked(const float* mass, const int32_t* seq_lens, int batch,
+                                  int row_stride, int k, const int32_t* exclude_cu,
+                                  const int32_t* exclude_slots, int32_t* tracked,
+                                  cudaStream_t stream);
+
+size_t step_bf16_smem_bytes();
+
+}  // namespace fdllm

@@ -1,0 +1,220 @@
+// Attention-mass reduction over heads and top-k tracking selection.
+//
+// "Flash-dLLM: I/O-Aware KV Caching and Parallel Decoding for Fast,
+// Memory-Efficient Diffusion LLMs" (ai4snews summary), paragraph 2: only a
+// fixed budget of the most-attended tokens is tracked and updated. The step
+// kernels write each head's per-key probability sums; this file turns them
+// into the per-sequence mass (mean over heads and rows, summed in a fixed
+// head order so the result is reproducible bit for bit) and selects the k
+// slots of largest mass.
+#include <cstdint>
+
+#include "fdllm_internal.h"
+
+namespace fdllm {
+namespace {
+
+__global__ void mass_reduce_kernel(const __grid_constant__ StepPlan plan, const float* part,
+                                   float* mass, int n_heads) {
+  const int b = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= plan.row_stride) return;
+  const int n = plan.cu_rows[b + 1] - plan.cu_rows[b];
+  float s = 0.f;
+  if (n > 0) {
+    const size_t hs = (size_t)plan.batch * plan.row_stride;
+    const float* p = part + (size_t)b * plan.row_stride + j;
+    for (int h = 0; h < n_heads; ++h) s += p[h * hs];
+    s *= 1.0f / (float)(n * n_heads);
+  }
+  mass[(size_t)b * plan.row_stride + j] = s;
+}
+
+// Order-preserving map of a float to an unsigned key (larger float, larger key).
+__device__ __forceinline__ uint32_t fkey(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+constexpr int SEL_THREADS = 1024;
+constexpr int SEL_MAXK = 1024;
+constexpr int SEL_MAXL = 65536;
+
+// One CTA per sequence. Exact radix select of the k-th largest key (4 passes
+// of 8 bits), then the strictly larger keys plus the lowest-slot ties, then a
+// bitonic sort by (key descending, slot ascending).
+__global__ void __launch_bounds__(SEL_THREADS)
+    select_kernel(const float* mass, const int32_t* seq_lens, int row_stride, int k,
+                  const int32_t* exclude_cu, const int32_t* exclude_slots, int32_t* tracked) {
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const float* m = mass + (size_t)b * row_stride;
+  int L = seq_lens[b];
+  if (L < 0) L = 0;
+  if (L > row_stride) L = row_stride;
+
+  __shared__ uint32_t excl[SEL_MAXL / 32];
+  __shared__ int hist[256];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining;
+  __shared__ int s_total;
+  __shared__ int s_cnt;
+  __shared__ int s_eqbase;
+  __shared__ uint32_t sk[SEL_MAXK];
+  __shared__ int ss[SEL_MAXK];
+  __shared__ int warp_sums[SEL_THREADS / 32];
+
+  for (int i = tid; i < (L + 31) / 32; i += SEL_THREADS) excl[i] = 0u;
+  __syncthreads();
+  if (exclude_cu) {
+    const int e0 = exclude_cu[b], e1 = exclude_cu[b + 1];
+    for (int e = e0 + tid; e < e1; e += SEL_THREADS) {
+      const int s = exclude_slots[e];
+      if (s >= 0 && s < L) atomicOr(&excl[s >> 5], 1u << (s & 31));
+    }
+  }
+  if (tid == 0) s_total = 0;
+  __syncthreads();
+  // candidate count
+  {
+    int c = 0;
+    for (int j = tid; j < L; j += SEL_THREADS) c += ((excl[j >> 5] >> (j & 31)) & 1u) ? 0 : 1;
+    atomicAdd(&s_total, c);
+  }
+  __syncthreads();
+  const int total = s_total;
+  const int want = total < k ? total : k;
+
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = want;
+  if (want > 0 && want < total) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
+      __syncthreads();
+      for (int j = tid; j < L; j += SEL_THREADS) {
+        if ((excl[j >> 5] >> (j & 31)) & 1u) continue;
+        const uint32_t key = fkey(m[j]);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, d = 255;
+        for (; d > 0; --d) {
+          if (cum + hist[d] >= remaining) break;
+          cum += hist[d];
+        }
+        s_prefix = prefix | ((uint32_t)d << shift);
+        s_remaining = remaining - cum;
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      remaining = s_remaining;
+      pmask |= 255u << shift;
+      __syncthreads();
+    }
+  }
+  // threshold key T = prefix (when want < total); take every key > T and the
+  // `remaining` lowest slots with key == T.
+  const bool all = (want == total);
+  if (tid == 0) s_cnt = 0;
+  __syncthreads();
+  for (int j = tid; j < L; j += SEL_THREADS) {
+    if ((excl[j >> 5] >> (j & 31)) & 1u) continue;
+    const uint32_t key = fkey(m[j]);
+    if (all || key > prefix) {
+      const int p = atomicAdd(&s_cnt, 1);
+      sk[p] = key;
+      ss[p] = j;
+    }
+  }
+  __syncthreads();
+  if (!all && remaining > 0) {
+    // ties at the threshold, lowest slots first: block-wide scan in slot order
+    if (tid == 0) s_eqbase = 0;
+    __syncthreads();
+    for (int base = 0; base < L; base += SEL_THREADS) {
+      const int j = base + tid;
+      int f = 0;
+      if (j < L && !((excl[j >> 5] >> (j & 31)) & 1u) && fkey(m[j]) == prefix) f = 1;
+      // inclusive scan of f across the block
+      int v = f;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, v, o);
+        if ((tid & 31) >= o) v += t;
+      }
+      if ((tid & 31) == 31) warp_sums[tid >> 5] = v;
+      __syncthreads();
+      if (tid < 32) {
+        int w = warp_sums[tid];
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, w, o);
+          if (tid >= o) w += t;
+        }
+        warp_sums[tid] = w;
+      }
+      __syncthreads();
+      const int excl_before = (tid >= 32 ? warp_sums[(tid >> 5) - 1] : 0) + v - f;
+      const int rank = s_eqbase + excl_before;
+      if (f && rank < remaining) {
+        const int p = (want - remaining) + rank;
+        sk[p] = prefix;
+        ss[p] = j;
+      }
+      __syncthreads();
+      if (tid == 0) s_eqbase += warp_sums[SEL_THREADS / 32 - 1];
+      __syncthreads();
+      if (s_eqbase >= remaining) break;
+    }
+  }
+  __syncthreads();
+  // pad and sort by (key desc, slot asc)
+  int P2 = 1;
+  while (P2 < want) P2 <<= 1;
+  for (int i = want + tid; i < P2; i += SEL_THREADS) {
+    sk[i] = 0u;
+    ss[i] = 0x7fffffff;
+  }
+  __syncthreads();
+  for (int size = 2; size <= P2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < P2; i += SEL_THREADS) {
+        const int jx = i ^ stride;
+        if (jx > i) {
+          const bool up = (i & size) == 0;   // "up" = descending by (key, -slot)
+          const uint32_t ka = sk[i], kb = sk[jx];
+          const int sa = ss[i], sb = ss[jx];
+          const bool a_first = (ka > kb) || (ka == kb && sa < sb);
+          if (up ? !a_first : a_first) {
+            sk[i] = kb;
+            sk[jx] = ka;
+            ss[i] = sb;
+            ss[jx] = sa;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < k; i += SEL_THREADS)
+    tracked[(size_t)b * k + i] = (i < want) ? ss[i] : -1;
+}
+
+}  // namespace
+
+cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
+                               cudaStream_t stream) {
+  dim3 grid((plan.row_stride + 255) / 256, plan.batch);
+  mass_reduce_kernel<<<grid, 256, 0, stream>>>(plan, part, mass, n_heads);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_tracked(const float* mass, const int32_t* seq_lens, int batch,
+                                  int row_stride, int k, const int32_t* exclude_cu,
+                                  const int32_t* exclude_slots, int32_t* tracked,
+                                  cudaStream_t stream) {
+  select_kernel<<<batch, SEL_THREADS, 0, stream>>>(mass, seq_lens, row_stride, k, exclude_cu,
+                                                   exclude_slots, tracked);
+  return cudaGetLastError();
+}
+
+}  // namespace fdllm

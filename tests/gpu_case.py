@@ -1,0 +1,140 @@
+"""Shared helpers for the GPU parity tests: run one seeded step through the
+C-ABI library and through the CPU oracle, and compare them.
+
+Tolerances (the spec bar):
+  * out: max |gpu - oracle| <= 1e-2 * RMS(oracle out)  (bf16 inputs, fp32
+    accumulation); fp32 workloads use 1e-4.
+  * attn_mass: |gpu - oracle| <= 1e-3 * |oracle| + 1e-6.
+  * cache: every byte outside the written slots bit-identical to the
+    pre-state; written slots within 1 bf16 ulp of the oracle or within
+    1e-2 * RMS of the written tensor (fp32: 1e-5 relative).
+  * tracked top-k: identical to the oracle's selection on the same fp32
+    mass; against the oracle's own mass, identical except at near-ties
+    (relative gap <= 1e-3).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import kv_cache_attention_flash_b200 as fd
+from kv_cache_attention_flash_b200 import workloads as W
+from oracle import oracle as O
+
+
+@dataclasses.dataclass
+class GpuRun:
+    out: np.ndarray
+    mass: np.ndarray
+    tracked: np.ndarray
+    k_pool: np.ndarray      # bits of the layer slice after the step
+    v_pool: np.ndarray
+
+
+def written_mask(meta, shape):
+    """[num_pages, page_size] bool: slots the step writes."""
+    ps = shape.page_size
+    m = np.zeros((meta.num_pages, ps), bool)
+    for b in range(meta.batch):
+        for r in range(meta.cu_rows[b], meta.cu_rows[b + 1]):
+            s = int(meta.slots[r])
+            m[meta.block_table[b, s // ps], s % ps] = True
+    return m
+
+
+def build_inputs(spec, seed=0, device="cpu", meta=None):
+    meta = meta if meta is not None else W.make_meta(spec, seed)
+    x = W.make_x(spec, meta, seed, device=device)
+    w = W.make_w(spec, seed, device=device)
+    kp, vp = W.make_pools(spec, meta, seed, device=device, n_layers=1)
+    return meta, x, w, kp, vp
+
+
+def run_gpu(spec, meta, x, w, kp, vp, layer=0, with_mass=True, validate=True, cache=None):
+    sh = spec.shape
+    dev = "cuda"
+    kp_d = kp.to(dev).contiguous()
+    vp_d = vp.to(dev).contiguous()
+    own = cache is None
+    if own:
+        cache = fd.FlashCache(kp_d.shape[0], sh.n_heads, sh.head_dim, sh.page_size, meta.num_pages,
+                              meta.max_position, sh.rope_theta, sh.dtype, max_batch=meta.batch,
+                              max_slots_per_seq=meta.max_blocks * sh.page_size,
+                              k_pool=kp_d, v_pool=vp_d)
+    pos = torch.from_numpy(meta.positions).to(dev)
+    slots = torch.from_numpy(meta.slots).to(dev)
+    view = torch.from_numpy(meta.view).to(dev)
+    bt = torch.from_numpy(meta.block_table).to(dev)
+    out, mass = cache.step(layer, meta.cu_rows, meta.seq_lens, x.to(dev), w.to(dev), pos, bt,
+                           view_mask=view, slots=slots, with_mass=with_mass, validate=validate)
+    cache.check()
+    tracked = None
+    if with_mass:
+        sl = torch.from_numpy(meta.seq_lens).to(dev)
+        ecu = torch.from_numpy(meta.exclude_cu).to(dev)
+        esl = torch.from_numpy(meta.exclude_slots if len(meta.exclude_slots) else np.zeros(1, np.int32)).to(dev)
+        tracked = fd.fdllm_select_tracked(mass, sl, meta.track_k, ecu, esl).cpu().numpy()
+    torch.cuda.synchronize()
+    res = GpuRun(out.cpu().numpy(), mass.cpu().numpy() if with_mass else None, tracked,
+                 W.bits_np(cache.k_pool[layer]), W.bits_np(cache.v_pool[layer]))
+    if own:
+        cache.close()
+    return res
+
+
+def run_oracle(spec, meta, x, w, kp, vp):
+    return O.layer_step(spec.shape, W.bits_np(kp), W.bits_np(vp), 0, W.bits_np(x), W.bits_np(w),
+                        meta.positions, meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table,
+                        meta.view)
+
+
+def tol_out(spec):
+    return 1e-2 if spec.shape.dtype == "bf16" else 1e-4
+
+
+def compare(spec, meta, gpu: GpuRun, orc, kp_pre_bits, vp_pre_bits):
+    o_out, o_mass, o_kp, o_vp = orc
+    sh = spec.shape
+    # out
+    rms = float(np.sqrt(np.mean(o_out ** 2)))
+    err = float(np.max(np.abs(gpu.out - o_out)))
+    assert np.all(np.isfinite(gpu.out)), "non-finite output"
+    assert err <= tol_out(spec) * rms, f"out: max err {err:.3e} > {tol_out(spec)} * rms {rms:.3e}"
+    # cache bytes
+    wm = written_mask(meta, sh)
+    full = np.broadcast_to(wm[:, None, :, None], gpu.k_pool.shape)
+    for name, g, pre, orv in (("k", gpu.k_pool, kp_pre_bits[0], o_kp[0]),
+                              ("v", gpu.v_pool, vp_pre_bits[0], o_vp[0])):
+        assert np.array_equal(g[~full], pre[~full]), f"{name}: bytes outside written slots changed"
+        gv = O.decode(g[full], sh.dtype)
+        ov = O.decode(orv[full], sh.dtype)
+        assert np.all(np.isfinite(gv)), f"{name}: a written slot holds a non-finite value"
+        if sh.dtype == "bf16":
+            ulp = np.abs(O.round_to_bf16(ov * (1 + 2.0 ** -8)) - ov) + 1e-30
+            wrms = float(np.sqrt(np.mean(ov ** 2)))
+            bad = (np.abs(gv - ov) > 1.01 * ulp) & (np.abs(gv - ov) > 1e-2 * wrms)
+        else:
+            bad = np.abs(gv - ov) > 1e-5 * (np.abs(ov) + np.sqrt(np.mean(ov ** 2)))
+        assert not np.any(bad), f"{name}: {int(bad.sum())} written values off"
+    # mass
+    if gpu.mass is not None:
+        mdiff = np.abs(gpu.mass - o_mass)
+        assert np.all(mdiff <= 1e-3 * np.abs(o_mass) + 1e-6), f"mass: max diff {mdiff.max():.3e}"
+        # selection: exact on the same fp32 input
+        ex_cu = meta.exclude_cu
+        ex = meta.exclude_slots
+        same = O.select_tracked(gpu.mass, meta.seq_lens, meta.track_k, ex_cu, ex)
+        assert np.array_equal(gpu.tracked, same), "select_tracked differs from the oracle on the same mass"
+        # against the oracle's own mass: near-ties only
+        ref = O.select_tracked(o_mass, meta.seq_lens, meta.track_k, ex_cu, ex)
+        for b in range(meta.batch):
+            a_set = set(gpu.tracked[b][gpu.tracked[b] >= 0].tolist())
+            b_set = set(ref[b][ref[b] >= 0].tolist())
+            if a_set == b_set:
+                continue
+            kth = min(o_mass[b, j] for j in b_set)
+            for j in a_set ^ b_set:
+                assert abs(o_mass[b, j] - kth) <= 1e-3 * kth, f"seq {b}: slot {j} is not a near-tie"
+    return err / max(rms, 1e-30)

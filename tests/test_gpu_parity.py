@@ -1,0 +1,195 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+the same seeded inputs. Small cases span several tiles and ragged tails; the
+full-size cases are the five layer workloads (the 32-layer stack is checked
+on sampled layers)."""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_attention_flash_b200 as fd
+from kv_cache_attention_flash_b200 import workloads as W
+from oracle import oracle as O
+
+from gpu_case import build_inputs, compare, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["small_bf16_divergent", "small_bf16_two_view", "small_f32_divergent",
+                                  "tiny_f32"])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_parity_small(name, seed):
+    spec = W.get_spec(name)
+    meta, x, w, kp, vp = build_inputs(spec, seed)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp))
+
+
+@pytest.mark.parametrize("name", ["llada8b_b1", "b32_divergent", "two_view_b8"])
+def test_parity_full_size(name):
+    spec = W.get_spec(name)
+    meta, x, w, kp, vp = build_inputs(spec, 0)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp))
+
+
+def test_parity_without_mass_output():
+    spec = W.get_spec("small_bf16_divergent")
+    meta, x, w, kp, vp = build_inputs(spec, 3)
+    g = run_gpu(spec, meta, x, w, kp, vp, with_mass=False)
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    rms = np.sqrt(np.mean(o[0] ** 2))
+    assert np.max(np.abs(g.out - o[0])) <= 1e-2 * rms
+
+
+def test_block_table_permutation_is_bitwise_invariant():
+    spec = W.get_spec("small_bf16_divergent")
+    meta, x, w, kp, vp = build_inputs(spec, 4)
+    g1 = run_gpu(spec, meta, x, w, kp, vp)
+    rng = np.random.default_rng(99)
+    perm = rng.permutation(meta.num_pages)
+    kp2 = torch.empty_like(kp)
+    vp2 = torch.empty_like(vp)
+    kp2[:, torch.from_numpy(perm)] = kp
+    vp2[:, torch.from_numpy(perm)] = vp
+    import dataclasses
+    meta2 = dataclasses.replace(meta, block_table=np.where(meta.block_table >= 0,
+                                                           perm[np.maximum(meta.block_table, 0)], -1).astype(np.int32))
+    g2 = run_gpu(spec, meta2, x, w, kp2, vp2)
+    assert np.array_equal(g1.out, g2.out)
+    assert np.array_equal(g1.mass, g2.mass)
+    assert np.array_equal(g1.tracked, g2.tracked)
+
+
+def test_two_views_isolated_bitwise_on_gpu():
+    spec = W.get_spec("small_bf16_two_view")
+    meta, x, w, kp, vp = build_inputs(spec, 5)
+    g1 = run_gpu(spec, meta, x, w, kp, vp)
+    x2 = x.clone()
+    mrows = torch.from_numpy(np.nonzero(meta.view == 2)[0])
+    x2[mrows] = torch.randn(len(mrows), x.shape[1]).to(x.dtype)
+    g2 = run_gpu(spec, meta, x2, w, kp, vp)
+    d = meta.view == 1
+    assert np.array_equal(g1.out[d], g2.out[d])
+    assert not np.array_equal(g1.out[~d], g2.out[~d])
+
+
+def test_select_tracked_matches_oracle_exactly():
+    rng = np.random.default_rng(7)
+    for trial in range(6):
+        B = int(rng.integers(1, 9))
+        stride = int(rng.choice([64, 300, 1024, 4096, 9000]))
+        k = int(rng.choice([1, 8, 32, 64, 200, 1024]))
+        lens = rng.integers(0, stride + 1, B).astype(np.int32)
+        # many exact ties: values on a coarse grid
+        mass = (rng.integers(0, 50, (B, stride)) / 997.0).astype(np.float32)
+        if trial % 2:
+            mass = rng.random((B, stride)).astype(np.float32)
+        ex = [rng.choice(max(int(L), 1), size=min(int(L), 5), replace=False) if L else np.zeros(0, int) for L in lens]
+        ex_cu = np.zeros(B + 1, np.int32)
+        ex_cu[1:] = np.cumsum([len(e) for e in ex])
+        ex_s = np.concatenate(ex).astype(np.int32) if ex_cu[-1] else np.zeros(1, np.int32)
+        dev = "cuda"
+        got = fd.fdllm_select_tracked(torch.from_numpy(mass).to(dev), torch.from_numpy(lens).to(dev), k,
+                                      torch.from_numpy(ex_cu).to(dev), torch.from_numpy(ex_s).to(dev)).cpu().numpy()
+        ref = O.select_tracked(mass, lens, k, ex_cu, ex_s)
+        assert np.array_equal(got, ref), trial
+
+
+def test_device_bounds_errors_are_reported_not_trapped():
+    spec = W.get_spec("small_bf16_divergent")
+    meta, x, w, kp, vp = build_inputs(spec, 6)
+    import dataclasses
+    bt = meta.block_table.copy()
+    bt[1, 0] = meta.num_pages + 5          # a context page outside the pool
+    bad = dataclasses.replace(meta, block_table=bt)
+    with pytest.raises(fd.FdllmError) as e:
+        run_gpu(spec, bad, x, w, kp, vp, validate=False)
+    assert e.value.status == 4
+    pos = meta.positions.copy()
+    pos[3] = 10 ** 6                        # outside the RoPE table
+    bad = dataclasses.replace(meta, positions=pos)
+    with pytest.raises(fd.FdllmError) as e:
+        run_gpu(spec, bad, x, w, kp, vp, validate=False)
+    assert e.value.status == 4
+    # validate mode catches it on the host before launching
+    with pytest.raises(fd.FdllmError) as e:
+        run_gpu(spec, bad, x, w, kp, vp, validate=True)
+    assert e.value.status == 1
+    # the handle stays usable after an error: a clean step still matches
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp))
+
+
+def test_edge_cases_empty_and_maximal_sequences():
+    """Sequences with no rows, a sequence with the maximum 128 rows, a
+    context shorter than one page, and a view-only sequence with no context."""
+    sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
+    spec = W.WorkloadSpec("edge", sh, batch=4, kind="divergent", ctx_min=1, ctx_max=1)
+    rng = np.random.default_rng(11)
+    lens = np.array([300, 0, 40, 0], np.int32)
+    rows = []
+    # seq 0: 128 plain rows inside its context
+    p0 = np.sort(rng.choice(300, 128, replace=False))
+    rows.append((p0, p0, np.zeros(128, np.int8)))
+    # seq 1: no rows at all
+    rows.append((np.zeros(0, int), np.zeros(0, int), np.zeros(0, np.int8)))
+    # seq 2: 5 plain rows, short context (less than one page)
+    p2 = np.sort(rng.choice(40, 5, replace=False))
+    rows.append((p2, p2, np.zeros(5, np.int8)))
+    # seq 3: two views of 3 rows, no context
+    pv = np.arange(0, 3)
+    rows.append((np.concatenate([pv, pv]), np.concatenate([pv, pv + 3]),
+                 np.concatenate([np.ones(3, np.int8), np.full(3, 2, np.int8)])))
+    ps = sh.page_size
+    need = [300, 0, 40, 6]
+    nblk = [max(1, (n + ps - 1) // ps) for n in need]
+    npg = sum(nblk) + 2
+    perm = rng.permutation(npg)
+    bt = np.full((4, max(nblk)), -1, np.int32)
+    k = 0
+    for b in range(4):
+        for i in range(nblk[b]):
+            bt[b, i] = perm[k]
+            k += 1
+    cu = np.zeros(5, np.int32)
+    cu[1:] = np.cumsum([len(r[0]) for r in rows])
+    meta = W.StepMeta(batch=4, cu_rows=cu, seq_lens=lens,
+                      positions=np.concatenate([r[0] for r in rows]).astype(np.int32),
+                      slots=np.concatenate([r[1] for r in rows]).astype(np.int32),
+                      view=np.concatenate([r[2] for r in rows]).astype(np.int8), block_table=bt,
+                      num_pages=npg, max_position=400, exclude_cu=np.zeros(5, np.int32),
+                      exclude_slots=np.zeros(0, np.int32), track_k=8, stage=np.zeros(4, np.int8))
+    x = W.make_x(spec, meta, 1)
+    w = W.make_w(spec, 1)
+    kp, vp = W.make_pools(spec, meta, 1, n_layers=1)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp))
+    assert np.all(g.mass[1] == 0) and np.all(g.tracked[1] == -1)
+    assert np.allclose(g.mass[[0, 2, 3]].sum(1), 1.0, atol=1e-5)
+
+
+def test_all_rows_empty_step():
+    sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
+    spec = W.WorkloadSpec("empty", sh, batch=2, kind="divergent", ctx_min=1, ctx_max=1)
+    meta = W.StepMeta(batch=2, cu_rows=np.zeros(3, np.int32), seq_lens=np.array([10, 70], np.int32),
+                      positions=np.zeros(0, np.int32), slots=np.zeros(0, np.int32), view=np.zeros(0, np.int8),
+                      block_table=np.array([[0, -1], [1, 2]], np.int32), num_pages=3, max_position=100,
+                      exclude_cu=np.zeros(3, np.int32), exclude_slots=np.zeros(0, np.int32), track_k=4,
+                      stage=np.zeros(2, np.int8))
+    cache = fd.FlashCache(1, 2, 128, 64, 3, 100, 1e4, "bf16", 2, 128)
+    mass = torch.full((2, 128), 7.0, device="cuda")
+    out = torch.empty(0, 256, device="cuda")
+    fd.fdllm_layer_step(cache.handle, 0, meta.cu_rows, meta.seq_lens, 2,
+                        torch.empty(0, 256, dtype=torch.bfloat16, device="cuda"),
+                        torch.empty(256, 768, dtype=torch.bfloat16, device="cuda"),
+                        torch.empty(0, dtype=torch.int32, device="cuda"),
+                        torch.from_numpy(meta.block_table).cuda(), None, out, mass)
+    cache.check()
+    assert fd.fdllm_last_launch_count() == 1
+    assert torch.all(mass == 0)
+    cache.close()
