@@ -1,0 +1,456 @@
+"""Benchmark of the Flash-dLLM per-layer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the fused layer step (projection, RoPE, cache write, scheduled attention,
+attention mass) for every layer of the workload, then the top-k tracking
+selection. The default workload is the batch-32 divergent-length layer
+(32 sequences, context U[256, 1024], half caching stage, half update stage,
+LLaDA-8B layer shape, bf16).
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
+events on the launching stream with an L2 flush (a 256 MB write) between
+steps, outside the events; barrier + synchronize on both sides; the total is
+the max over ranks. Under torchrun each rank runs its own batch (independent
+sequences: weak scaling, no collective on the data path).
+
+One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kv_cache_attention_flash_b200 import workloads as W  # noqa: E402
+
+METRIC = "fused layer-step query-tokens/s; achieved HBM GB/s and % of roofline (1×B200)"
+UNIT = "query-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        self.window = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for t, line in self.samples:
+            if self.window and not (self.window[0] - 0.05 <= t <= self.window[1] + 0.05):
+                continue
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            rows.append(p)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ workload
+class Workload:
+    """Device-resident inputs of one workload (one rank's batch)."""
+
+    def __init__(self, name: str, seed: int, device):
+        import kv_cache_attention_flash_b200 as fd
+        self.fd = fd
+        self.spec = W.get_spec(name)
+        self.meta = W.make_meta(self.spec, seed)
+        sh = self.spec.shape
+        self.n_layers = sh.n_layers
+        self.device = device
+        m = self.meta
+        self.x = [W.make_x(self.spec, m, seed, layer=l, device=device) for l in range(self.n_layers)]
+        self.w = [W.make_w(self.spec, seed, layer=l, device=device) for l in range(self.n_layers)]
+        kp, vp = W.make_pools(self.spec, m, seed, device=device)
+        self.cache = fd.FlashCache(self.n_layers, sh.n_heads, sh.head_dim, sh.page_size, m.num_pages,
+                                   m.max_position, sh.rope_theta, sh.dtype, m.batch,
+                                   m.max_blocks * sh.page_size, k_pool=kp, v_pool=vp)
+        self.pos = torch.from_numpy(m.positions).to(device)
+        self.slots = torch.from_numpy(m.slots).to(device)
+        self.view = torch.from_numpy(m.view).to(device)
+        self.bt = torch.from_numpy(m.block_table).to(device)
+        self.seq_lens_d = torch.from_numpy(m.seq_lens).to(device)
+        self.ex_cu = torch.from_numpy(m.exclude_cu).to(device)
+        ex = m.exclude_slots if len(m.exclude_slots) else np.zeros(1, np.int32)
+        self.ex_sl = torch.from_numpy(ex).to(device)
+        R = m.total_rows
+        H = sh.hidden
+        self.out = torch.empty(R, H, dtype=torch.float32, device=device)
+        self.mass = torch.empty(m.batch, m.max_blocks * sh.page_size, dtype=torch.float32, device=device)
+        self.tracked = torch.empty(m.batch, m.track_k, dtype=torch.int32, device=device)
+        self.launches_per_step = None
+
+    def step(self, x_list=None, ev=None):
+        """One pass of the hot path; returns the number of kernels launched.
+        If `ev` is given, events are recorded around each layer step."""
+        fd = self.fd
+        m = self.meta
+        n = 0
+        xs = x_list if x_list is not None else self.x
+        for l in range(self.n_layers):
+            if ev is not None:
+                ev[0].record()
+            fd.fdllm_layer_step(self.cache.handle, l, m.cu_rows, m.seq_lens, m.max_blocks, xs[l],
+                                self.w[l], self.pos, self.bt, self.view, self.out, self.mass,
+                                self.slots)
+            if ev is not None:
+                ev[1].record()
+                ev = None
+            n += fd.fdllm_last_launch_count()
+        fd.fdllm_select_tracked(self.mass, self.seq_lens_d, m.track_k, self.ex_cu, self.ex_sl,
+                                self.tracked)
+        n += fd.fdllm_last_launch_count()
+        return n
+
+
+# ------------------------------------------------------------------ CPU baseline
+_ORACLE_INPUTS = {}
+
+
+def oracle_inputs(spec, meta, seed):
+    key = (spec.name, seed)
+    if key not in _ORACLE_INPUTS:
+        x = W.make_x(spec, meta, seed)
+        w = W.make_w(spec, seed)
+        kp, vp = W.make_pools(spec, meta, seed, n_layers=1)
+        _ORACLE_INPUTS[key] = (W.bits_np(x), W.bits_np(w), W.bits_np(kp), W.bits_np(vp))
+    return _ORACLE_INPUTS[key]
+
+
+def oracle_sample(spec, meta, seed, budget_s=12.0):
+    """Times the CPU oracle on a bounded sample of the workload: the first
+    sequences of layer 0 (as many as fit the time budget). Returns
+    (rows/s, description, threads)."""
+    sys.path.insert(0, ROOT)
+    from oracle import oracle as O
+    xb, wb, kb, vb = oracle_inputs(spec, meta, seed)
+    total_rows = 0
+    total_t = 0.0
+    nseq = 0
+    b = 0
+    while b < meta.batch and total_t < budget_s:
+        r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
+        cu = np.array([0, r1 - r0], np.int32)
+        t0 = time.perf_counter()
+        O.layer_step(spec.shape, kb, vb, 0, xb[r0:r1], wb, meta.positions[r0:r1], meta.slots[r0:r1], cu,
+                     meta.seq_lens[b:b + 1], meta.block_table[b:b + 1], meta.view[r0:r1])
+        total_t += time.perf_counter() - t0
+        total_rows += r1 - r0
+        nseq += 1
+        b += 1
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = (f"oracle (numpy float64) on {nseq} of {meta.batch} sequences of layer 0 "
+            f"({total_rows} query rows), one sequence per call, {total_t:.1f} s")
+    return total_rows / total_t, desc, threads
+
+
+def e2e_measure(wl: Workload, steps: int):
+    """Same metric through the public API with host buffers: per step the
+    inputs (x of every layer, positions, slots, views, block table) are copied
+    from pinned host memory, and out, attn_mass and the tracked set are read
+    back; all inside the timed region."""
+    fd = wl.fd
+    dev = wl.device
+    hx = [x.cpu().pin_memory() for x in wl.x]
+    hpos = wl.pos.cpu().pin_memory()
+    hslots = wl.slots.cpu().pin_memory()
+    hview = wl.view.cpu().pin_memory()
+    hbt = wl.bt.cpu().pin_memory()
+    dx = [torch.empty_like(x) for x in wl.x]
+    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    hmass = torch.empty(wl.mass.shape, dtype=wl.mass.dtype).pin_memory()
+    htr = torch.empty(wl.tracked.shape, dtype=wl.tracked.dtype).pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in hx) + sum(
+        t.numel() * t.element_size() for t in (hpos, hslots, hview, hbt))
+    d2h = sum(t.numel() * t.element_size() for t in (hout, hmass, htr))
+
+    def one():
+        for l in range(wl.n_layers):
+            dx[l].copy_(hx[l], non_blocking=True)
+        wl.pos.copy_(hpos, non_blocking=True)
+        wl.slots.copy_(hslots, non_blocking=True)
+        wl.view.copy_(hview, non_blocking=True)
+        wl.bt.copy_(hbt, non_blocking=True)
+        wl.step(x_list=dx)
+        hout.copy_(wl.out, non_blocking=True)
+        hmass.copy_(wl.mass, non_blocking=True)
+        htr.copy_(wl.tracked, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+# ------------------------------------------------------------------ main arms
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    spec = W.get_spec(args.workload)
+    meta = W.make_meta(spec, args.seed)
+    budget = max(2.0, 20.0 / max(1, args.steps + args.warmup))
+    vals = []
+    desc = ""
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        v, desc, threads = oracle_sample(spec, meta, args.seed, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(v)
+    value = float(np.mean(vals))
+    R = meta.total_rows * spec.shape.n_layers
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * R / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_block(spec, meta, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def config_block(spec, meta, args):
+    sh = spec.shape
+    return {"workload": spec.name, "layers": sh.n_layers, "batch": meta.batch,
+            "query_rows_per_layer": meta.total_rows,
+            "context_slots": [int(meta.seq_lens.min()), int(meta.seq_lens.max())],
+            "hidden": sh.hidden, "heads": sh.n_heads, "head_dim": sh.head_dim,
+            "page_size": sh.page_size, "track_k": meta.track_k,
+            "l2": "flushed between timed steps (256 MB write)", "parallelism": f"replicas x{args.gpus}",
+            "seed": args.seed}
+
+
+def run_native(args):
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    wl = Workload(args.workload, args.seed + rank, dev)
+    spec, meta = wl.spec, wl.meta
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    for _ in range(args.warmup):
+        wl.step()
+    wl.cache.check()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_ls = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_le = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev_s[i].record()
+        launches += wl.step(ev=(ev_ls[i], ev_le[i]))
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    if sampler:
+        sampler.mark(t_wall0, t_wall1)
+        time.sleep(0.25)
+        sampler.stop()
+    wl.cache.check()
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    layer_ms = [ev_ls[i].elapsed_time(ev_le[i]) for i in range(args.steps)]
+    total_ms_local = float(sum(step_ms))
+    total_ms = reduce_max(total_ms_local, dev)
+    rows_local = meta.total_rows * args.steps
+    rows_all = reduce_sum(rows_local, dev)
+    value = rows_all / (total_ms / 1000.0)
+
+    # roofline of the dominant kernel (the fused layer step, layer 0)
+    byt, fl = W.algorithmic_bytes_flops(spec, meta)
+    kern_s = float(np.mean(layer_ms)) / 1000.0
+    t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
+    t_tc = fl / (peaks["bf16_tflops"] * 1e12)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    if bound == "tensor":
+        achieved, peak, unit = fl / kern_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = byt / kern_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": args.traffic, "peak_source": f"{peak_src} (burst)",
+            "kernel": "fdllm_layer_step (fused step kernel + mass reduce), layer 0",
+            "kernel_us": kern_s * 1e6, "algorithmic_bytes": byt, "algorithmic_flops": fl,
+            "hbm_gbs_achieved": byt / kern_s / 1e9,
+            "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline": max(t_hbm, t_tc) / kern_s}
+
+    e2e_ms, h2d, d2h = e2e_measure(wl, max(10, min(args.steps, 200)))
+    e2e_val_local = meta.total_rows / (e2e_ms / 1000.0)
+    e2e_ms_max = reduce_max(e2e_ms, dev)
+    e2e_value = meta.total_rows * world / (e2e_ms_max / 1000.0)
+    del e2e_val_local
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads = oracle_sample(spec, meta, args.seed + rank)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    clocks = sampler.summary() if sampler else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": spec.shape.dtype, "data": "synthetic",
+        "config": config_block(spec, meta, argparse.Namespace(gpus=world, seed=args.seed)),
+        "layer_steps_per_s": value / meta.total_rows * spec.shape.n_layers,
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms_max},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    wl.cache.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="b32_divergent", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the step kernel, when captured for this build")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

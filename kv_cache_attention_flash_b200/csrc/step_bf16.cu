@@ -572,23 +572,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        // O += P V over the warp's KW keys, 16 keys per MMA step
+        // O += P V over the warp's KW keys, 16 keys per MMA step. P enters
+        // the tensor cores as bf16 hi + lo parts (P - hi rounded again), so
+        // the product carries ~16 significant bits of P; V is exact bf16.
         const uint8_t* vd = smem + KV_OFF + (c & 1) * KV_BUF + KC * D * 2;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (16 * u < KW) {
-            uint32_t pa[4];
-            pa[0] = ptx::pack_bf16(sacc[2 * u][0], sacc[2 * u][1]);
-            pa[1] = ptx::pack_bf16(sacc[2 * u][2], sacc[2 * u][3]);
-            pa[2] = ptx::pack_bf16(sacc[2 * u + 1][0], sacc[2 * u + 1][1]);
-            pa[3] = ptx::pack_bf16(sacc[2 * u + 1][2], sacc[2 * u + 1][3]);
+            uint32_t ph[4], pl[4];
+            ptx::split_bf16(sacc[2 * u][0], sacc[2 * u][1], ph[0], pl[0]);
+            ptx::split_bf16(sacc[2 * u][2], sacc[2 * u][3], ph[1], pl[1]);
+            ptx::split_bf16(sacc[2 * u + 1][0], sacc[2 * u + 1][1], ph[2], pl[2]);
+            ptx::split_bf16(sacc[2 * u + 1][2], sacc[2 * u + 1][3], ph[3], pl[3]);
             const int vrow = sp * KW + 16 * u + (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
             for (int dp = 0; dp < 8; ++dp) {
               uint32_t vb[4];
               ptx::ldmatrix_x4_trans(vb, vd + swz(vrow, 2 * dp + (lane >> 4)));
-              ptx::mma_bf16_16816(oacc[2 * dp], pa, vb);
-              ptx::mma_bf16_16816(oacc[2 * dp + 1], pa, vb + 2);
+              ptx::mma_bf16_16816(oacc[2 * dp], ph, vb);
+              ptx::mma_bf16_16816(oacc[2 * dp + 1], ph, vb + 2);
+              ptx::mma_bf16_16816(oacc[2 * dp], pl, vb);
+              ptx::mma_bf16_16816(oacc[2 * dp + 1], pl, vb + 2);
             }
           }
         }

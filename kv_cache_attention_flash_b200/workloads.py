@@ -243,6 +243,22 @@ def make_x(spec: WorkloadSpec, meta: StepMeta, seed: int, layer: int = 0,
     return x.to(torch_dtype(spec.shape))
 
 
+def make_x_onehot(spec: WorkloadSpec, meta: StepMeta, seed: int, scale: float = 64.0,
+                  device="cpu") -> torch.Tensor:
+    """x [R, H] whose rows are scale * e_i for seeded columns i (scale a power
+    of two). With it every projected value is one bf16 entry of Wqkv times a
+    power of two, so fp32 and fp64 accumulation give the same number and no
+    bf16 rounding decision can differ between two implementations. With
+    scale 64 and Wqkv ~ N(0, 0.02^2) the projected values are N(0, 1.28^2),
+    the magnitude of the dense workloads."""
+    rng = np.random.default_rng(seed * 7 + 3)
+    H = spec.shape.hidden
+    idx = rng.integers(0, H, meta.total_rows)
+    x = torch.zeros(meta.total_rows, H, dtype=torch.float32, device=device)
+    x[torch.arange(meta.total_rows, device=device), torch.from_numpy(idx).to(device)] = scale
+    return x.to(torch_dtype(spec.shape))
+
+
 def make_w(spec: WorkloadSpec, seed: int, layer: int = 0, device="cpu") -> torch.Tensor:
     """Wqkv [H, 3H] row-major, N(0, 0.02^2); columns are [Q | K | V], each
     block head-major (head h at columns h*D .. h*D+D-1)."""

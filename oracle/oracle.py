@@ -140,7 +140,7 @@ def visible_keys(L: int, view: np.ndarray, positions: np.ndarray, slots: np.ndar
 # --------------------------------------------------------------------------
 
 def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
-               cu_rows, seq_lens, block_table, view):
+               cu_rows, seq_lens, block_table, view, probs=None):
     """One Flash-Cache + scheduled-attention layer step.
 
     shape: object with dtype ("bf16"/"f32"), hidden, n_heads, head_dim,
@@ -154,6 +154,8 @@ def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
 
     Returns (out [R, H] float64, mass [B, max_blocks * page_size] float64,
              k_pool', v_pool').
+    If `probs` is a dict, probs[(b, h)] = (key slots, P [R_b, keys]) is
+    recorded for the tests' error analysis (no effect on the results).
 
     Steps [FD ¶1]: project the selected rows, rotate q and k, write k and v
     into the paged cache, then attend over each sequence's pages through its
@@ -161,18 +163,28 @@ def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
     tracked tokens; the per-key attention mass feeds the next tracked set.
     [FD ¶3]: the draft and mask views share positions (hence RoPE) and are
     isolated from each other."""
+    a = project(shape, x_bits, w_bits)
+    return layer_step_from_projection(shape, k_pool, v_pool, layer, a, positions, slots,
+                                      cu_rows, seq_lens, block_table, view, probs)
+
+
+def project(shape, x_bits, w_bits):
+    """Step 1, the QKV projection: a = x Wqkv in float64 (library matmul on
+    the exact values of the bf16/fp32 inputs). [R, 3H]."""
+    return decode(x_bits, shape.dtype) @ decode(w_bits, shape.dtype)
+
+
+def layer_step_from_projection(shape, k_pool, v_pool, layer, a, positions, slots, cu_rows,
+                               seq_lens, block_table, view, probs=None):
+    """Steps 2-6 of layer_step from a given projection result a [R, 3H]."""
     dt = shape.dtype
     H, nh, D, ps = shape.hidden, shape.n_heads, shape.head_dim, shape.page_size
     k_pool = k_pool.copy()
     v_pool = v_pool.copy()
-    x = decode(x_bits, dt)
-    w = decode(w_bits, dt)
     B = len(seq_lens)
-    R = x.shape[0]
+    R = a.shape[0]
     row_stride = block_table.shape[1] * ps
 
-    # 1. projection  (library matmul in float64)
-    a = x @ w                                            # [R, 3H]
     q = a[:, 0:H].reshape(R, nh, D)
     k = a[:, H:2 * H].reshape(R, nh, D)
     v = a[:, 2 * H:3 * H].reshape(R, nh, D)
@@ -207,6 +219,8 @@ def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
             S = (q[r0:r1, h, :] @ Kc[:, h, :].T) / np.sqrt(D)
             P = softmax_rows(S, vis)
             out[r0:r1, h * D:(h + 1) * D] = P @ Vc[:, h, :]
+            if probs is not None:
+                probs[(b, h)] = (keys, P)
             # 6. attention mass: mean over heads and rows  [FD ¶2]
             np.add.at(mass[b], keys, P.sum(axis=0) / ((r1 - r0) * nh))
     return out, mass, k_pool, v_pool

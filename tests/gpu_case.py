@@ -1,13 +1,27 @@
 """Shared helpers for the GPU parity tests: run one seeded step through the
 C-ABI library and through the CPU oracle, and compare them.
 
-Tolerances (the spec bar):
-  * out: max |gpu - oracle| <= 1e-2 * RMS(oracle out)  (bf16 inputs, fp32
-    accumulation); fp32 workloads use 1e-4.
+Tolerances. The spec bar for bf16 is max |out_gpu - out_oracle| <=
+1e-2 * RMS(out_oracle) (fp32 workloads: 1e-4), indexing bit-exact.
+
+  * mode "exact" (x rows one-hot times a power of two): the projection is
+    exact in fp32 and fp64 alike, so no bf16 rounding decision can differ.
+    out must meet the plain bar; written v must be bit-identical; written k
+    (rotated in fp32 on the GPU, fp64 in the oracle) within 1 bf16 ulp plus
+    1e-5 * RMS for values next to zero.
+  * mode "dense" (x ~ N(0,1)): the bf16 codes of the fresh q/k/v are decided
+    from an fp32 accumulator on the GPU and an fp64 one in the oracle; where
+    the two land on opposite sides of a rounding midpoint both codes are
+    correct. Written values: 1 bf16 ulp plus 1e-3 * RMS (the size of an fp32
+    accumulation error over K = 4096, which exceeds one ulp of values near
+    zero). out, per element: 1e-2 * RMS + sum over fresh keys of P * ulp(v)
+    (the largest effect of one-ulp changes of the fresh v, from the oracle's
+    own P and v) + 2 * the spread that the same fp32-vs-fp64 choice for q and
+    k alone produces inside the oracle (projection re-accumulated in float32
+    by numpy for the q and k columns).
   * attn_mass: |gpu - oracle| <= 1e-3 * |oracle| + 1e-6.
   * cache: every byte outside the written slots bit-identical to the
-    pre-state; written slots within 1 bf16 ulp of the oracle or within
-    1e-2 * RMS of the written tensor (fp32: 1e-5 relative).
+    pre-state.
   * tracked top-k: identical to the oracle's selection on the same fp32
     mass; against the oracle's own mass, identical except at near-ties
     (relative gap <= 1e-3).
@@ -84,24 +98,77 @@ def run_gpu(spec, meta, x, w, kp, vp, layer=0, with_mass=True, validate=True, ca
     return res
 
 
-def run_oracle(spec, meta, x, w, kp, vp):
+def run_oracle(spec, meta, x, w, kp, vp, probs=None):
     return O.layer_step(spec.shape, W.bits_np(kp), W.bits_np(vp), 0, W.bits_np(x), W.bits_np(w),
                         meta.positions, meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table,
-                        meta.view)
+                        meta.view, probs=probs)
+
+
+def qk_rounding_spread(spec, meta, x, w, kp, vp, o_out):
+    """max |out' - out| where out' re-accumulates the q and k columns of the
+    projection in float32 (a legitimate fp32 implementation's rounding
+    choices) and keeps everything else of the oracle."""
+    sh = spec.shape
+    H = sh.hidden
+    a = O.project(sh, W.bits_np(x), W.bits_np(w))
+    xf = O.decode(W.bits_np(x), sh.dtype).astype(np.float32)
+    wf = O.decode(W.bits_np(w), sh.dtype).astype(np.float32)
+    a[:, :2 * H] = (xf @ wf[:, :2 * H]).astype(np.float64)
+    alt = O.layer_step_from_projection(sh, W.bits_np(kp), W.bits_np(vp), 0, a, meta.positions,
+                                       meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table,
+                                       meta.view)[0]
+    return float(np.max(np.abs(alt - o_out)))
+
+
+def bf16_ulp(v):
+    """Spacing of bfloat16 numbers at |v| (normal range)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def fresh_v_sensitivity(spec, meta, probs, o_vp):
+    """Per output element: sum over this step's fresh keys j of
+    P_rj * ulp(v_j,d), the largest change a one-ulp change of every fresh v
+    can make."""
+    sh = spec.shape
+    D, ps = sh.head_dim, sh.page_size
+    R = meta.total_rows
+    t = np.zeros((R, sh.hidden))
+    for (b, h), (keys, P) in probs.items():
+        r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
+        fresh = set(int(s) for s in meta.slots[r0:r1])
+        sel = [i for i, k in enumerate(keys) if int(k) in fresh]
+        if not sel:
+            continue
+        ks = keys[sel]
+        pages = meta.block_table[b, ks // ps]
+        v = O.decode(o_vp[0, pages, h, ks % ps, :], sh.dtype)       # [nf, D]
+        t[r0:r1, h * D:(h + 1) * D] += P[:, sel] @ bf16_ulp(v)
+    return t
 
 
 def tol_out(spec):
     return 1e-2 if spec.shape.dtype == "bf16" else 1e-4
 
 
-def compare(spec, meta, gpu: GpuRun, orc, kp_pre_bits, vp_pre_bits):
+def compare(spec, meta, gpu: GpuRun, orc, kp_pre_bits, vp_pre_bits, mode="plain", probs=None,
+            qk_spread=0.0):
+    """mode: "exact" (one-hot x), "dense" (needs probs and qk_spread) or
+    "plain" (plain bound everywhere; fp32 workloads)."""
     o_out, o_mass, o_kp, o_vp = orc
     sh = spec.shape
     # out
     rms = float(np.sqrt(np.mean(o_out ** 2)))
-    err = float(np.max(np.abs(gpu.out - o_out)))
+    diff = np.abs(gpu.out - o_out)
+    err = float(np.max(diff))
     assert np.all(np.isfinite(gpu.out)), "non-finite output"
-    assert err <= tol_out(spec) * rms, f"out: max err {err:.3e} > {tol_out(spec)} * rms {rms:.3e}"
+    if mode != "dense" or sh.dtype != "bf16":
+        assert err <= tol_out(spec) * rms, f"out: max err {err:.3e} > {tol_out(spec)} * rms {rms:.3e}"
+    else:
+        extra = fresh_v_sensitivity(spec, meta, probs, o_vp)
+        bad = diff > tol_out(spec) * rms + extra + 2.0 * qk_spread
+        assert not np.any(bad), (f"out: {int(bad.sum())} elements over the dense bound; "
+                                 f"max err/rms {err / rms:.3e}, qk spread/rms {qk_spread / rms:.3e}")
     # cache bytes
     wm = written_mask(meta, sh)
     full = np.broadcast_to(wm[:, None, :, None], gpu.k_pool.shape)
@@ -111,13 +178,16 @@ def compare(spec, meta, gpu: GpuRun, orc, kp_pre_bits, vp_pre_bits):
         gv = O.decode(g[full], sh.dtype)
         ov = O.decode(orv[full], sh.dtype)
         assert np.all(np.isfinite(gv)), f"{name}: a written slot holds a non-finite value"
-        if sh.dtype == "bf16":
-            ulp = np.abs(O.round_to_bf16(ov * (1 + 2.0 ** -8)) - ov) + 1e-30
-            wrms = float(np.sqrt(np.mean(ov ** 2)))
-            bad = (np.abs(gv - ov) > 1.01 * ulp) & (np.abs(gv - ov) > 1e-2 * wrms)
+        wrms = float(np.sqrt(np.mean(ov ** 2))) if ov.size else 0.0
+        if sh.dtype != "bf16":
+            bad = np.abs(gv - ov) > 1e-5 * (np.abs(ov) + wrms)
+        elif mode == "exact" and name == "v":
+            bad = g[full] != orv[full]
+        elif mode == "exact":
+            bad = np.abs(gv - ov) > bf16_ulp(ov) * 1.0001 + 1e-5 * wrms
         else:
-            bad = np.abs(gv - ov) > 1e-5 * (np.abs(ov) + np.sqrt(np.mean(ov ** 2)))
-        assert not np.any(bad), f"{name}: {int(bad.sum())} written values off"
+            bad = np.abs(gv - ov) > bf16_ulp(ov) * 1.0001 + 1e-3 * wrms
+        assert not np.any(bad), f"{name}: {int(bad.sum())} written values off (mode {mode})"
     # mass
     if gpu.mass is not None:
         mdiff = np.abs(gpu.mass - o_mass)
