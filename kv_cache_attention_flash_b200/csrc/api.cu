@@ -73,6 +73,8 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 
 struct fdllm_cache {
   fdllm_cache_config cfg;
+  CUtensorMap tmap_k;   // pools viewed as [rows = layer/page/head/slot][head_dim] (bf16)
+  CUtensorMap tmap_v;
   void* k_pool;
   void* v_pool;
   int device;
@@ -124,11 +126,24 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
     return fail(FDLLM_ERR_UNSUPPORTED, "cache_create: fp32 kernel serves head_dim 32/64/96/128");
   if (c.max_batch > kMaxBatch)
     return fail(FDLLM_ERR_UNSUPPORTED, "cache_create: max_batch > %d", kMaxBatch);
+  if (c.dtype == FDLLM_BF16 && c.page_size != kBf16PageSize)
+    return fail(FDLLM_ERR_UNSUPPORTED, "cache_create: bf16 kernels gather %d-slot pages",
+                kBf16PageSize);
+  if ((long long)c.n_layers * c.num_pages * c.n_heads * c.page_size >= (1ll << 31))
+    return fail(FDLLM_ERR_UNSUPPORTED, "cache_create: pool has 2^31 or more slot rows");
 
   fdllm_cache* h = new fdllm_cache();
   h->cfg = c;
   h->k_pool = k_pool;
   h->v_pool = v_pool;
+  if (c.dtype == FDLLM_BF16) {
+    const uint64_t rows = (uint64_t)c.n_layers * c.num_pages * c.n_heads * c.page_size;
+    if (!encode_bf16_2d(&h->tmap_k, k_pool, rows, (uint64_t)c.head_dim, (uint32_t)c.page_size) ||
+        !encode_bf16_2d(&h->tmap_v, v_pool, rows, (uint64_t)c.head_dim, (uint32_t)c.page_size)) {
+      delete h;
+      return fail(FDLLM_ERR_CUDA, "cache_create: cuTensorMapEncodeTiled failed for the pools");
+    }
+  }
   cudaGetDevice(&h->device);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
@@ -277,6 +292,9 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   if (c.dtype == FDLLM_BF16) {
     if (H % 64)
       return fail(FDLLM_ERR_UNSUPPORTED, "layer_step: hidden %d not a multiple of 64", H);
+    if (st->max_blocks_per_seq > kBf16MaxPages)
+      return fail(FDLLM_ERR_UNSUPPORTED, "layer_step: more than %d pages per sequence",
+                  kBf16MaxPages);
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(wqkv)) & 15)
       return fail(FDLLM_ERR_INVALID_ARG, "layer_step: x and wqkv must be 16-byte aligned");
   }
@@ -297,18 +315,25 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   plan.layer = layer;
   for (int b = 0; b <= st->batch; ++b) plan.cu_rows[b] = st->cu_rows[b];
   for (int b = 0; b < st->batch; ++b) plan.seq_lens[b] = st->seq_lens[b];
-  // Pack whole sequences, in order, into groups of at most 128 rows.
-  int ng = 0, cur = 0;
+  // Pack whole sequences, in order, into groups of at most 128 rows. Inside
+  // a group each sequence's q rows start on a multiple of 16 (the attention
+  // MMA's N granularity), and the padded rows also fit in 128.
+  int ng = 0, cur = 0, cur_pad = 0;
   for (int b = 0; b < st->batch; ++b) {
     const int n = st->cu_rows[b + 1] - st->cu_rows[b];
+    const int n16 = (n + 15) & ~15;
+    plan.seq_qoff[b] = 0;
     if (n == 0) continue;
-    if (ng == 0 || cur + n > kGroupRows) {
+    if (ng == 0 || cur + n > kGroupRows || cur_pad + n16 > kGroupRows) {
       plan.group_row0[ng] = st->cu_rows[b];
       plan.group_seq0[ng] = (ng == 0) ? 0 : b;
       ++ng;
       cur = 0;
+      cur_pad = 0;
     }
+    plan.seq_qoff[b] = cur_pad;
     cur += n;
+    cur_pad += n16;
   }
   plan.group_row0[ng] = R;
   plan.group_seq0[ng] = st->batch;
@@ -343,7 +368,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
       if (!encode_bf16_2d(&tx, x, (uint64_t)R, (uint64_t)H, 128) ||
           !encode_bf16_2d(&tw, wqkv, (uint64_t)H, (uint64_t)3 * H, 64))
         return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed");
-      e = launch_step_bf16(plan, a, &tx, &tw, s);
+      e = launch_step_bf16(plan, a, &tx, &tw, &h->tmap_k, &h->tmap_v, s);
     } else {
       e = launch_step_f32(plan, a, s);
     }

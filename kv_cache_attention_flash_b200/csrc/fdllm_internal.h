@@ -10,6 +10,8 @@ constexpr int kMaxBatch = 256;        // sequences per step
 constexpr int kMaxGroups = 256;       // 128-row groups per step
 constexpr int kGroupRows = 128;       // rows per group (the MMA's M)
 constexpr int kMaxSeqRows = 128;      // rows per sequence
+constexpr int kBf16PageSize = 64;     // page size of the bf16 kernel's page gathers
+constexpr int kBf16MaxPages = 512;    // logical pages per sequence (bf16 kernel)
 
 // Device error word layout (int32[4]).
 enum DevErr : int {
@@ -32,6 +34,7 @@ struct StepPlan {
   int group_seq0[kMaxGroups + 1];  // group g: sequences [group_seq0[g], group_seq0[g+1])
   int cu_rows[kMaxBatch + 1];
   int seq_lens[kMaxBatch];
+  int seq_qoff[kMaxBatch];         // first q row of the sequence in its group (multiple of 16)
 };
 
 // Per-call device pointers and pool geometry.
@@ -59,7 +62,8 @@ struct StepArgs {
 
 // Launchers (return cudaGetLastError()).
 cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* tmap_x,
-                             const void* tmap_w, cudaStream_t stream);
+                             const void* tmap_w, const void* tmap_k, const void* tmap_v,
+                             cudaStream_t stream);
 cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
                                cudaStream_t stream);
