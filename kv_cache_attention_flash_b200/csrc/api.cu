@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <set>
 #include <string>
 #include <vector>
@@ -64,6 +65,25 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Wqkv [H][3H] bf16 viewed in 5 dimensions (column c within a 64-column
+// half, K row k, half, q/k/v block, head): element (c, k, half, blk, head)
+// is Wqkv[k][blk * H + head * head_dim + half * 64 + c]. One box
+// {64, 64, 2, 3, 1} is one head's q, k and v columns for 64 K rows, written
+// to shared memory as six 8 KB [64 rows][128 B] sub-boxes (128-byte swizzle).
+bool encode_wqkv_5d(CUtensorMap* map, const void* base, uint64_t hidden, uint64_t n_heads,
+                    uint64_t head_dim) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[5] = {64, hidden, head_dim / 64, 3, n_heads};
+  cuuint64_t strides[4] = {3 * hidden * 2, 128, hidden * 2, head_dim * 2};
+  cuuint32_t box[5] = {64, 64, (cuuint32_t)(head_dim / 64), 3, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -315,29 +335,63 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   plan.layer = layer;
   for (int b = 0; b <= st->batch; ++b) plan.cu_rows[b] = st->cu_rows[b];
   for (int b = 0; b < st->batch; ++b) plan.seq_lens[b] = st->seq_lens[b];
-  // Pack whole sequences, in order, into groups of at most 128 rows. Inside
-  // a group each sequence's q rows start on a multiple of 16 (the attention
-  // MMA's N granularity), and the padded rows also fit in 128.
-  int ng = 0, cur = 0, cur_pad = 0;
-  for (int b = 0; b < st->batch; ++b) {
-    const int n = st->cu_rows[b + 1] - st->cu_rows[b];
-    const int n16 = (n + 15) & ~15;
-    plan.seq_qoff[b] = 0;
-    if (n == 0) continue;
-    if (ng == 0 || cur + n > kGroupRows || cur_pad + n16 > kGroupRows) {
-      plan.group_row0[ng] = st->cu_rows[b];
-      plan.group_seq0[ng] = (ng == 0) ? 0 : b;
-      ++ng;
-      cur = 0;
-      cur_pad = 0;
+  // Row groups (one 128-row tile each): whole sequences, each padded to a
+  // multiple of 16 q rows (the attention MMA's N granularity), packed first
+  // fit in order of decreasing size. The bf16 kernel also keeps a group's
+  // attended page list on chip (at most kBf16GroupPages entries, bounded by
+  // context pages + rows). Groups are then ordered by decreasing attention
+  // work so that the costliest tiles start first.
+  {
+    struct Grp {
+      int pad, pages;
+      long long cost;
+      std::vector<int> seqs;
+    };
+    std::vector<int> idx;
+    for (int b = 0; b < st->batch; ++b) {
+      plan.seq_qoff[b] = 0;
+      if (st->cu_rows[b + 1] > st->cu_rows[b]) idx.push_back(b);
     }
-    plan.seq_qoff[b] = cur_pad;
-    cur += n;
-    cur_pad += n16;
+    auto n16 = [&](int b) { return (st->cu_rows[b + 1] - st->cu_rows[b] + 15) & ~15; };
+    auto pages = [&](int b) {
+      return (st->seq_lens[b] + c.page_size - 1) / c.page_size + st->cu_rows[b + 1] - st->cu_rows[b];
+    };
+    std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
+      if (n16(x) != n16(y)) return n16(x) > n16(y);
+      return st->seq_lens[x] > st->seq_lens[y];
+    });
+    std::vector<Grp> groups;
+    for (int b : idx) {
+      Grp* dst = nullptr;
+      for (auto& gp : groups)
+        if (gp.pad + n16(b) <= kGroupRows && gp.pages + pages(b) <= kBf16GroupPages &&
+            (int)gp.seqs.size() < kGroupRows / 16) {
+          dst = &gp;
+          break;
+        }
+      if (!dst) {
+        groups.push_back(Grp{0, 0, 0, {}});
+        dst = &groups.back();
+      }
+      plan.seq_qoff[b] = dst->pad;
+      dst->pad += n16(b);
+      dst->pages += pages(b);
+      dst->cost += (long long)(st->seq_lens[b] + c.page_size) * n16(b);
+      dst->seqs.push_back(b);
+    }
+    if ((int)groups.size() > kMaxGroups)
+      return fail(FDLLM_ERR_UNSUPPORTED, "layer_step: more than %d row groups", kMaxGroups);
+    std::stable_sort(groups.begin(), groups.end(),
+                     [](const Grp& x, const Grp& y) { return x.cost > y.cost; });
+    int k = 0;
+    for (size_t gi = 0; gi < groups.size(); ++gi) {
+      plan.group_seq0[gi] = k;
+      for (int b : groups[gi].seqs) plan.seq_order[k++] = b;
+    }
+    plan.group_seq0[groups.size()] = k;
+    plan.n_groups = (int)groups.size();
   }
-  plan.group_row0[ng] = R;
-  plan.group_seq0[ng] = st->batch;
-  plan.n_groups = ng;
+  const int ng = plan.n_groups;
 
   StepArgs a;
   a.x = x;
@@ -364,11 +418,16 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   cudaError_t e = cudaSuccess;
   if (ng > 0) {
     if (c.dtype == FDLLM_BF16) {
-      CUtensorMap tx, tw;
-      if (!encode_bf16_2d(&tx, x, (uint64_t)R, (uint64_t)H, 128) ||
-          !encode_bf16_2d(&tw, wqkv, (uint64_t)H, (uint64_t)3 * H, 64))
-        return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed");
-      e = launch_step_bf16(plan, a, &tx, &tw, &h->tmap_k, &h->tmap_v, s);
+      CUtensorMap tx[4], tw;
+      const void* txp[4];
+      for (int i = 0; i < 4; ++i) {
+        if (!encode_bf16_2d(&tx[i], x, (uint64_t)R, (uint64_t)H, 16u << i))
+          return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (x)");
+        txp[i] = &tx[i];
+      }
+      if (!encode_wqkv_5d(&tw, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim))
+        return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv)");
+      e = launch_step_bf16(plan, a, txp, &tw, &h->tmap_k, &h->tmap_v, s);
     } else {
       e = launch_step_f32(plan, a, s);
     }

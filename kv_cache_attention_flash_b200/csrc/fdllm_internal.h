@@ -12,6 +12,7 @@ constexpr int kGroupRows = 128;       // rows per group (the MMA's M)
 constexpr int kMaxSeqRows = 128;      // rows per sequence
 constexpr int kBf16PageSize = 64;     // page size of the bf16 kernel's page gathers
 constexpr int kBf16MaxPages = 512;    // logical pages per sequence (bf16 kernel)
+constexpr int kBf16GroupPages = 1024; // attended pages per row group (bf16 kernel)
 
 // Device error word layout (int32[4]).
 enum DevErr : int {
@@ -30,11 +31,12 @@ struct StepPlan {
   int max_blocks;        // block table row length
   int row_stride;        // max_blocks * page_size (mass row length)
   int layer;
-  int group_row0[kMaxGroups + 1];  // group g: rows [group_row0[g], group_row0[g+1])
-  int group_seq0[kMaxGroups + 1];  // group g: sequences [group_seq0[g], group_seq0[g+1])
+  int group_seq0[kMaxGroups + 1];  // group g: sequences seq_order[group_seq0[g] .. group_seq0[g+1])
+  int seq_order[kMaxBatch];        // sequences with rows, group by group
   int cu_rows[kMaxBatch + 1];
   int seq_lens[kMaxBatch];
-  int seq_qoff[kMaxBatch];         // first q row of the sequence in its group (multiple of 16)
+  int seq_qoff[kMaxBatch];         // first q row of the sequence in its group's 128-row tile
+                                   // (a multiple of 16)
 };
 
 // Per-call device pointers and pool geometry.
@@ -61,7 +63,8 @@ struct StepArgs {
 };
 
 // Launchers (return cudaGetLastError()).
-cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* tmap_x,
+// tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
+cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* const* tmap_x,
                              const void* tmap_w, const void* tmap_k, const void* tmap_v,
                              cudaStream_t stream);
 cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream);

@@ -31,6 +31,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstddef>
+
 #include "fdllm_internal.h"
 #include "ptx.cuh"
 
@@ -47,9 +49,14 @@ constexpr int B_BYTES = 6 * BOX_BYTES;         // q, k, v blocks, two boxes each
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES; // 64 KB
 constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
 constexpr int TMEM_COLS = 512;
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 320;        // warps 0-7: epilogue / softmax (two per TMEM quadrant),
+                                      // warp 8: TMA producer, warp 9: MMA issuer and TMEM owner
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int NSMX = 256;             // threads of warps 0-7
 constexpr int PS = 64;                          // cache page size served
-constexpr int MAX_PAGES = 512;                  // logical pages per sequence
+constexpr int MAX_PAGES = 1024;                 // logical pages attended per row group
+constexpr int MAX_SEQ = 8;                      // sequences per row group (16 padded rows each)
 constexpr uint64_t WAIT_NS = 1000000000ull;     // bounded waits: 1 s
 
 // Reuse of the pipeline area after the projection.
@@ -86,15 +93,20 @@ struct Ctrl {
   int row_page[BM];       // -1: row has bad metadata
   int row_view[BM];
   int row_q[BM];          // row of q in shared memory (sequences padded to 16 rows)
-  // current sequence
-  int nx, npages;
-  int xs_slot[BM];        // slots written by view rows, ascending
-  int xs_row[BM];         // their group rows
-  int pg_log[MAX_PAGES];  // logical pages attended, in order
-  int pg_phys[MAX_PAGES]; // physical page, -1 when the table entry is bad
-  float m_run[BM], l_run[BM], mnew[BM], lse2[BM];
-  float red[4][BM];
+  int row_seq[BM];        // sequence (index into sq_*) of each row
+  // sequences of the group that have rows (each takes >= 16 padded q rows)
+  int nseq;
+  int sq_b[MAX_SEQ], sq_n[MAX_SEQ], sq_L[MAX_SEQ], sq_gr0[MAX_SEQ], sq_qoff[MAX_SEQ];
+  int sq_npages[MAX_SEQ], sq_pg0[MAX_SEQ], sq_x0[MAX_SEQ], sq_nx[MAX_SEQ], sq_any[MAX_SEQ];
+  int xs_slot[BM];        // per sequence: slots written by its view rows, ascending
+  int xs_row[BM];         //   and the group rows that write them
+  short pg_log[MAX_PAGES];  // per sequence: logical pages attended, in order
+  int pg_phys[MAX_PAGES];   //   and their physical pages (-1: bad table entry)
+  alignas(16) float lse2[BM];   // log2-sum-exp2 of the scaled scores of each row (float4 loads)
+  float pm[BM], pl[BM];          // pass-1 partial (max, sum) of the second key half
 };
+static_assert(offsetof(Ctrl, lse2) % 16 == 0, "lse2 is read as float4");
+static_assert(sizeof(Ctrl) % 16 == 0 || true, "");
 constexpr int CTRL_OFF = PIPE_BYTES;
 constexpr int SMEM_BYTES = PIPE_BYTES + (int)sizeof(Ctrl) + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -131,24 +143,6 @@ __device__ __forceinline__ void named_bar(int id, int n) {
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Reduce-scatter of 32 columns over the 32 lanes: afterwards v[0] of lane l
-// holds the max (or sum) over all lanes of column l.
-template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(float* v, int lane) {
-#pragma unroll
-  for (int k = 16; k >= 1; k >>= 1) {
-    const bool upper = (lane & k) != 0;
-#pragma unroll
-    for (int i = 0; i < k; ++i) {
-      const float send = upper ? v[i] : v[i + k];
-      const float keep = upper ? v[i + k] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, k);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  return v[0];
 }
 
 __device__ __forceinline__ void rope32(float* lo, float* hi, int pos, int c, const float* cos_t,
@@ -219,7 +213,10 @@ __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     step_bf16_kernel(const __grid_constant__ StepPlan plan, const __grid_constant__ StepArgs a,
-                     const __grid_constant__ CUtensorMap tmap_x,
+                     const __grid_constant__ CUtensorMap tmap_x16,
+                     const __grid_constant__ CUtensorMap tmap_x32,
+                     const __grid_constant__ CUtensorMap tmap_x64,
+                     const __grid_constant__ CUtensorMap tmap_x128,
                      const __grid_constant__ CUtensorMap tmap_w,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
@@ -233,8 +230,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int lane = tid & 31;
   const int h = blockIdx.x / plan.n_groups;
   const int g = blockIdx.x % plan.n_groups;
-  const int row0 = plan.group_row0[g];
-  const int nrows = plan.group_row0[g + 1] - row0;
+  // sequences of this group: plan.seq_order[seq_a .. seq_b); sequence b
+  // owns q rows [seq_qoff[b], seq_qoff[b] + n_b) of the 128-row tile, which
+  // are also the TMEM lanes of the projection
   const int seq_a = plan.group_seq0[g];
   const int seq_b = plan.group_seq0[g + 1];
   const int H = a.hidden;
@@ -252,21 +250,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&ctrl->s_full[s], 1);
-      ptx::mbar_init(&ctrl->s_empty[s], 4);
+      ptx::mbar_init(&ctrl->s_empty[s], 8);
     }
     ptx::mbar_init(&ctrl->mma_done, 1);
-    ptx::mbar_init(&ctrl->p_full, 4);
+    ptx::mbar_init(&ctrl->p_full, 8);
     ptx::mbar_init(&ctrl->pv_done, 1);
     ptx::mbar_init(&ctrl->o_done, 1);
     ctrl->abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     ptx::tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (tid == 64) {
-    ptx::prefetch_tmap(&tmap_x);
+  if (warp == kProducerWarp && lane == 1) {
+    ptx::prefetch_tmap(&tmap_x16);
+    ptx::prefetch_tmap(&tmap_x32);
+    ptx::prefetch_tmap(&tmap_x64);
+    ptx::prefetch_tmap(&tmap_x128);
     ptx::prefetch_tmap(&tmap_w);
     ptx::prefetch_tmap(&tmap_k);
     ptx::prefetch_tmap(&tmap_v);
@@ -277,24 +278,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = ctrl->tmem_base;
 
   // ================================================================ projection
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {   // TMA producer
+      // x boxes of the tile, computed once: each sequence's (16-padded) rows
+      // in the largest boxes that fit (at most 8 boxes for 128 rows)
+      int nbox = 0, x_rows = 0;
+      uint32_t box_dst[8];
+      int box_row[8], box_h[8];
+      for (int q = seq_a; q < seq_b; ++q) {
+        const int b = plan.seq_order[q];
+        int rem = (plan.cu_rows[b + 1] - plan.cu_rows[b] + 15) & ~15;
+        int off = 0;
+        x_rows += rem;
+        while (rem > 0 && nbox < 8) {
+          const int hgt = rem >= 128 ? 128 : rem >= 64 ? 64 : rem >= 32 ? 32 : 16;
+          box_dst[nbox] = (uint32_t)(plan.seq_qoff[b] + off) * 128u;
+          box_row[nbox] = plan.cu_rows[b] + off;
+          box_h[nbox] = hgt;
+          ++nbox;
+          off += hgt;
+          rem -= hgt;
+        }
+      }
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % STAGES;
         const int u = kb / STAGES;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
         uint8_t* st = smem + s * STAGE_BYTES;
-        ptx::mbar_arrive_expect_tx(&ctrl->full[s], STAGE_BYTES);
-        ptx::tma_load_2d(st, &tmap_x, kb * BK, row0, &ctrl->full[s]);
+        ptx::mbar_arrive_expect_tx(&ctrl->full[s], B_BYTES + x_rows * BK * 2);
 #pragma unroll
-        for (int blk = 0; blk < 3; ++blk)
-#pragma unroll
-          for (int half = 0; half < 2; ++half)
-            ptx::tma_load_2d(st + A_BYTES + (blk * 2 + half) * BOX_BYTES, &tmap_w,
-                             blk * H + h * D + half * 64, kb * BK, &ctrl->full[s]);
+        for (int i = 0; i < 8; ++i) {
+          if (i < nbox) {
+            const CUtensorMap* mx = box_h[i] == 128 ? &tmap_x128 : box_h[i] == 64 ? &tmap_x64
+                                  : box_h[i] == 32 ? &tmap_x32 : &tmap_x16;
+            ptx::tma_load_2d(st + box_dst[i], mx, kb * BK, box_row[i], &ctrl->full[s]);
+          }
+        }
+        // this head's q, k and v column blocks of Wqkv, two 64-column halves
+        // each: one 48 KB box of the 5-D view (column, K row, half, block,
+        // head), laid out as six [64 K rows][64 columns] sub-boxes
+        ptx::tma_load_5d(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s]);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {   // MMA issuer
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, 128, false, true);
       for (int kb = 0; kb < nkb; ++kb) {
@@ -322,17 +348,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ptx::umma_commit(&ctrl->mma_done);
     }
   } else {
-    // row metadata (warps 2..7)
-    for (int i = tid - 64; i < BM; i += NTHREADS - 64) {
-      int pos = 0, slot = 0, page = -1, view = 0, qr = 0;
-      if (i < nrows) {
-        const int gr = row0 + i;
+    // ---- group metadata, built by warps 0..7 while the projection runs
+    const int mt = tid;
+    constexpr int NM = NSMX;
+    if (mt == 0) {
+      int ns = 0;
+      for (int q = seq_a; q < seq_b; ++q) {
+        const int b = plan.seq_order[q];
+        const int n = plan.cu_rows[b + 1] - plan.cu_rows[b];
+        if (n == 0 || ns >= MAX_SEQ) continue;
+        ctrl->sq_b[ns] = b;
+        ctrl->sq_n[ns] = n;
+        ctrl->sq_L[ns] = plan.seq_lens[b];
+        ctrl->sq_gr0[ns] = plan.cu_rows[b];
+        ctrl->sq_qoff[ns] = plan.seq_qoff[b];
+        ++ns;
+      }
+      ctrl->nseq = ns;
+    }
+    named_bar(2, NM);
+    const int nseq = ctrl->nseq;
+    // q rows of the tile: position, slot, page, view, sequence
+    for (int i = mt; i < BM; i += NM) {
+      int pos = 0, slot = 0, page = -1, view = 0, qr = i, sq = -1;
+      for (int q = 0; q < nseq; ++q)
+        if (i >= ctrl->sq_qoff[q] && i < ctrl->sq_qoff[q] + ctrl->sq_n[q]) sq = q;
+      if (sq >= 0) {
+        const int gr = ctrl->sq_gr0[sq] + (i - ctrl->sq_qoff[sq]);
+        const int b = ctrl->sq_b[sq];
         pos = a.positions[gr];
         slot = a.slots ? a.slots[gr] : pos;
         view = a.view ? (int)a.view[gr] : 0;
-        int b = seq_a;
-        while (b + 1 < seq_b && plan.cu_rows[b + 1] <= gr) ++b;
-        qr = plan.seq_qoff[b] + (gr - plan.cu_rows[b]);
         if (pos < 0 || pos >= a.max_position) {
           set_err(a.err, kDevBadPosition, gr);
         } else if (slot < 0 || slot >= plan.row_stride) {
@@ -350,6 +396,108 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ctrl->row_page[i] = page;
       ctrl->row_view[i] = view;
       ctrl->row_q[i] = qr;
+      ctrl->row_seq[i] = sq;
+    }
+    named_bar(2, NM);
+    // view rows with good metadata, per sequence
+    if (mt < nseq) {
+      int c = 0;
+      for (int i = ctrl->sq_qoff[mt]; i < ctrl->sq_qoff[mt] + ctrl->sq_n[mt]; ++i)
+        c += (ctrl->row_view[i] != 0 && ctrl->row_page[i] >= 0) ? 1 : 0;
+      ctrl->sq_nx[mt] = c;
+    }
+    named_bar(2, NM);
+    if (mt == 0) {
+      int x = 0;
+      for (int q = 0; q < nseq; ++q) {
+        ctrl->sq_x0[q] = x;
+        x += ctrl->sq_nx[q];
+      }
+    }
+    named_bar(2, NM);
+    // view slots of each sequence, ascending (rank sort)
+    for (int i = mt; i < BM; i += NM) {
+      if (ctrl->row_seq[i] < 0 || ctrl->row_view[i] == 0 || ctrl->row_page[i] < 0) continue;
+      const int q = ctrl->row_seq[i];
+      const int si = ctrl->row_slot[i];
+      int rank = 0;
+      for (int j = ctrl->sq_qoff[q]; j < ctrl->sq_qoff[q] + ctrl->sq_n[q]; ++j) {
+        if (ctrl->row_view[j] == 0 || ctrl->row_page[j] < 0) continue;
+        const int sj = ctrl->row_slot[j];
+        rank += (sj < si || (sj == si && j < i)) ? 1 : 0;
+      }
+      ctrl->xs_slot[ctrl->sq_x0[q] + rank] = si;
+      ctrl->xs_row[ctrl->sq_x0[q] + rank] = i;
+    }
+    named_bar(2, NM);
+    // logical pages: the context pages, then the pages of view slots past them
+    if (mt < nseq) {
+      const int npr = (ctrl->sq_L[mt] + PS - 1) / PS;
+      int np = npr, last = -1;
+      for (int t = 0; t < ctrl->sq_nx[mt]; ++t) {
+        const int p = ctrl->xs_slot[ctrl->sq_x0[mt] + t] / PS;
+        if (p >= npr && p != last) {
+          ++np;
+          last = p;
+        }
+      }
+      ctrl->sq_npages[mt] = np;
+    }
+    named_bar(2, NM);
+    if (mt == 0) {
+      int o = 0;
+      for (int q = 0; q < nseq; ++q) {
+        ctrl->sq_pg0[q] = o;
+        if (o + ctrl->sq_npages[q] > MAX_PAGES) {
+          set_err(a.err, kDevBadSlot, -2);
+          ctrl->sq_npages[q] = MAX_PAGES - o;
+        }
+        o += ctrl->sq_npages[q];
+      }
+    }
+    named_bar(2, NM);
+    for (int q = 0; q < nseq; ++q) {
+      const int npr = min((ctrl->sq_L[q] + PS - 1) / PS, ctrl->sq_npages[q]);
+      const int* bt = a.block_table + (size_t)ctrl->sq_b[q] * plan.max_blocks;
+      for (int i = mt; i < npr; i += NM) {
+        const int pg = bt[i];
+        const bool ok = pg >= 0 && pg < a.num_pages;
+        if (!ok) set_err(a.err, kDevBadPage, -1 - i);
+        ctrl->pg_log[ctrl->sq_pg0[q] + i] = (short)i;
+        ctrl->pg_phys[ctrl->sq_pg0[q] + i] = ok ? pg : -1;
+      }
+    }
+    if (mt < nseq) {
+      const int q = mt;
+      const int npr = (ctrl->sq_L[q] + PS - 1) / PS;
+      const int* bt = a.block_table + (size_t)ctrl->sq_b[q] * plan.max_blocks;
+      int np = npr, last = -1;
+      for (int t = 0; t < ctrl->sq_nx[q] && np < ctrl->sq_npages[q]; ++t) {
+        const int p = ctrl->xs_slot[ctrl->sq_x0[q] + t] / PS;
+        if (p >= npr && p != last) {
+          const int pg = bt[p];
+          const bool ok = pg >= 0 && pg < a.num_pages;
+          if (!ok) set_err(a.err, kDevBadPage, -1 - p);
+          ctrl->pg_log[ctrl->sq_pg0[q] + np] = (short)p;
+          ctrl->pg_phys[ctrl->sq_pg0[q] + np] = ok ? pg : -1;
+          ++np;
+          last = p;
+        }
+      }
+    }
+    named_bar(2, NM);
+    if (mt < nseq) {
+      int any = 0;
+      for (int i = 0; i < ctrl->sq_npages[mt]; ++i) any |= ctrl->pg_phys[ctrl->sq_pg0[mt] + i] >= 0;
+      ctrl->sq_any[mt] = any;
+    }
+    // mass partials: zero (the softmax warps accumulate into them)
+    if (a.mass_part) {
+      for (int q = 0; q < nseq; ++q) {
+        float4* part = reinterpret_cast<float4*>(
+            a.mass_part + ((size_t)h * plan.batch + ctrl->sq_b[q]) * plan.row_stride);
+        for (int j = mt; j < plan.row_stride / 4; j += NM) part[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
   }
   __syncwarp();
@@ -362,10 +510,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   {
     const int quad = warp & 3;
     const int i = quad * 32 + lane;
-    const bool valid = acc_ok && i < nrows && ctrl->row_page[i] >= 0;
+    const bool valid = acc_ok && ctrl->row_page[i] >= 0;
     const int pos = ctrl->row_pos[i];
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-    if (warp < 4) {
+    if (warp >= 8) {
+      // producer and MMA warps take no part in the epilogue
+    } else if (warp < 4) {
       epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
     } else {
       epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF);
@@ -380,7 +530,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const size_t head_stride = (size_t)PS * D;
     __nv_bfloat16* kp = reinterpret_cast<__nv_bfloat16*>(a.k_pool);
     __nv_bfloat16* vp = reinterpret_cast<__nv_bfloat16*>(a.v_pool);
-    for (int idx = tid; idx < nrows * 32; idx += NTHREADS) {
+    for (int idx = tid; idx < BM * 32; idx += NTHREADS) {
       const int r = idx >> 5;
       const int part = idx & 31;
       const int ch = part & 15;
@@ -411,113 +561,84 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // issued so far, S^T products, P.V products, finished sequences.
   uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0;
 
-  for (int b = seq_a; b < seq_b; ++b) {
-    const int n = plan.cu_rows[b + 1] - plan.cu_rows[b];
-    if (n == 0) continue;
-    const int ra = plan.cu_rows[b] - row0;
-    const int L = plan.seq_lens[b];
+  const int nseq_g = ctrl->nseq;
+  for (int si = 0; si < nseq_g; ++si) {
+    const int b = ctrl->sq_b[si];
+    const int n = ctrl->sq_n[si];
+    const int ra = ctrl->sq_qoff[si];           // first q row (row metadata index)
+    const int gr0 = ctrl->sq_gr0[si];           // first row in x / out
+    const int L = ctrl->sq_L[si];
     const int N16 = (n + 15) & ~15;
-    const int qoff = plan.seq_qoff[b];
+    const int qoff = ctrl->sq_qoff[si];
     const int nblk = (N16 + 31) >> 5;
-
-    // ---------------------------------------- sequence setup (all threads)
-    // view rows with good metadata, sorted by slot
-    if (tid < n) {
-      const int i = ra + tid;
-      if (ctrl->row_view[i] != 0 && ctrl->row_page[i] >= 0) {
-        const int si = ctrl->row_slot[i];
-        int rank = 0;
-        for (int j = 0; j < n; ++j) {
-          const int jj = ra + j;
-          if (ctrl->row_view[jj] == 0 || ctrl->row_page[jj] < 0) continue;
-          const int sj = ctrl->row_slot[jj];
-          rank += (sj < si || (sj == si && j < tid)) ? 1 : 0;
-        }
-        ctrl->xs_slot[rank] = si;
-        ctrl->xs_row[rank] = i;
-      }
-    }
-    const int nx = __syncthreads_count(tid < n && ctrl->row_view[ra + tid] != 0 &&
-                                       ctrl->row_page[ra + tid] >= 0);
-    const int npr = min((L + PS - 1) / PS, MAX_PAGES);
-    for (int i = tid; i < npr; i += NTHREADS) ctrl->pg_log[i] = i;
-    if (tid == 0) {
-      int np = npr;
-      int last = -1;
-      for (int t = 0; t < nx; ++t) {
-        const int p = ctrl->xs_slot[t] / PS;
-        if (p >= npr && p != last && np < MAX_PAGES) {
-          ctrl->pg_log[np++] = p;
-          last = p;
-        }
-      }
-      ctrl->npages = np;
-    }
-    __syncthreads();
-    const int npages = ctrl->npages;
-    const int* bt = a.block_table + (size_t)b * plan.max_blocks;
-    for (int i = tid; i < npages; i += NTHREADS) {
-      const int pg = bt[ctrl->pg_log[i]];
-      if (pg < 0 || pg >= a.num_pages) {
-        set_err(a.err, kDevBadPage, -1 - ctrl->pg_log[i]);
-        ctrl->pg_phys[i] = -1;
-      } else {
-        ctrl->pg_phys[i] = pg;
-      }
-    }
-    if (tid < BM) {
-      ctrl->m_run[tid] = -INFINITY;
-      ctrl->l_run[tid] = 0.f;
-    }
-    __syncthreads();
+    const int npages = ctrl->sq_npages[si];
+    const int nx = ctrl->sq_nx[si];
+    const bool any_page = ctrl->sq_any[si] != 0;
+    const short* pgl = ctrl->pg_log + ctrl->sq_pg0[si];
+    const int* pgp = ctrl->pg_phys + ctrl->sq_pg0[si];
+    const int* xsl = ctrl->xs_slot + ctrl->sq_x0[si];
+    const int* xsr = ctrl->xs_row + ctrl->sq_x0[si];
     const int nch = (npages + 1) >> 1;
-    bool any_page = false;
-    for (int i = 0; i < npages; ++i) any_page |= ctrl->pg_phys[i] >= 0;
     float* part = a.mass_part ? a.mass_part + ((size_t)h * plan.batch + b) * plan.row_stride
                               : nullptr;
-    // Chunk loads of this sequence: pass 1 K_0..K_{nch-1} (items r0 + c),
-    // pass 2 K_c, V_c (items r0 + nch + 2c, r0 + nch + 2c + 1).
+    // Chunk loads of this sequence, in ring order: pass 1 K_0 .. K_{nch-1}
+    // (items r0 + c); pass 2 K_0, K_1, then V_c followed by K_{c+2}, so that
+    // K runs one chunk ahead of V and each load's slot was freed by a
+    // product issued a chunk earlier.
     const uint32_t r0 = ring, s0 = scount, p0 = pcount;
+    const int npre = nch < 2 ? nch : 2;
+    const int nk2 = nch > 2 ? nch - 2 : 0;
+    auto item_v2 = [&](int c) -> uint32_t {
+      return r0 + nch + npre + c + (c < nk2 ? c : nk2);
+    };
+    auto item_k2 = [&](int c) -> uint32_t { return c < 2 ? r0 + nch + c : item_v2(c - 2) + 1; };
 
-    if (warp == 0) {
+    if (warp == kProducerWarp) {
       // ---------------------------------------- TMA producer
       if (lane == 0) {
         uint32_t item = r0;
-        for (int pass = 0; pass < 2; ++pass) {
-          for (int c = 0; c < nch; ++c) {
-            for (int which = 0; which <= pass; ++which, ++item) {
-              const int s = item % NSLOT;
-              const uint32_t u = item / NSLOT;
-              if (u > 0) wait_bar(ctrl, &ctrl->aempty[s], (u - 1) & 1, a.err, 10);
-              uint32_t bytes = 0;
-              int phys[2] = {-1, -1};
-              for (int pi = 0; pi < 2; ++pi) {
-                const int pidx = 2 * c + pi;
-                if (pidx < npages && ctrl->pg_phys[pidx] >= 0) {
-                  phys[pi] = ctrl->pg_phys[pidx];
-                  bytes += 2 * BOX_BYTES;
-                }
-              }
-              ptx::mbar_arrive_expect_tx(&ctrl->afull[s], bytes);
-              uint8_t* dst = smem + SLOT_OFF + s * SLOT_BYTES;
-              const CUtensorMap* map = which == 0 ? &tmap_k : &tmap_v;
-              for (int pi = 0; pi < 2; ++pi) {
-                if (phys[pi] < 0) continue;
-                const int row = ((layer * a.num_pages + phys[pi]) * a.n_heads + h) * PS;
-                ptx::tma_load_2d(dst + pi * BOX_BYTES, map, 0, row, &ctrl->afull[s]);
-                ptx::tma_load_2d(dst + HALF_BYTES + pi * BOX_BYTES, map, 64, row, &ctrl->afull[s]);
-              }
+        auto load = [&](int c, bool is_v) {
+          const int s = item % NSLOT;
+          const uint32_t u = item / NSLOT;
+          if (u > 0) wait_bar(ctrl, &ctrl->aempty[s], (u - 1) & 1, a.err, 10);
+          uint32_t bytes = 0;
+          int phys[2] = {-1, -1};
+          for (int pi = 0; pi < 2; ++pi) {
+            const int pidx = 2 * c + pi;
+            if (pidx < npages && pgp[pidx] >= 0) {
+              phys[pi] = pgp[pidx];
+              bytes += 2 * BOX_BYTES;
             }
           }
+          ptx::mbar_arrive_expect_tx(&ctrl->afull[s], bytes);
+          uint8_t* dst = smem + SLOT_OFF + s * SLOT_BYTES;
+          const CUtensorMap* map = is_v ? &tmap_v : &tmap_k;
+          for (int pi = 0; pi < 2; ++pi) {
+            if (phys[pi] < 0) continue;
+            const int row = ((layer * a.num_pages + phys[pi]) * a.n_heads + h) * PS;
+            ptx::tma_load_2d(dst + pi * BOX_BYTES, map, 0, row, &ctrl->afull[s]);
+            ptx::tma_load_2d(dst + HALF_BYTES + pi * BOX_BYTES, map, 64, row, &ctrl->afull[s]);
+          }
+          ++item;
+        };
+        for (int c = 0; c < nch; ++c) load(c, false);
+        for (int c = 0; c < npre; ++c) load(c, false);
+        for (int c = 0; c < nch; ++c) {
+          load(c, true);
+          if (c + 2 < nch) load(c + 2, false);
         }
       }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
       // ---------------------------------------- MMA issuer
       if (lane == 0) {
+        const uint32_t idesc_std = ptx::idesc_bf16_f32(128, 128, false, false);
         const uint32_t idesc_s = ptx::idesc_bf16_f32(128, N16, false, false);
         const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, N16, true, true);
-        // S^T number j of this sequence from chunk-load item `item`.
-        auto issue_s = [&](uint32_t j, uint32_t item) {
+        // Score product number j of this sequence from chunk-load `item`:
+        // pass 1 S = Q K^T (rows of the whole group on lanes, keys on
+        // columns), pass 2 S^T = K Q^T (keys on lanes, this sequence's rows
+        // on columns).
+        auto issue_s = [&](uint32_t j, uint32_t item, bool transposed) {
           const int s = item % NSLOT;
           wait_bar(ctrl, &ctrl->afull[s], (item / NSLOT) & 1, a.err, 11);
           const uint32_t idx = s0 + j;
@@ -528,20 +649,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            // A: K chunk, K-major, M = 128 keys; B: q rows, K-major, N = N16.
-            const uint64_t ad = ptx::smem_desc_sw128(kbase + off, 16, 1024);
-            const uint64_t bd = ptx::smem_desc_sw128(q_base + off + qoff * 128, 16, 1024);
-            ptx::umma_f16_ss(tmem + (sb ? TM_S1 : TM_S0), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            // K chunk and q rows, both K-major 128-byte swizzled.
+            const uint64_t kd = ptx::smem_desc_sw128(kbase + off, 16, 1024);
+            if (transposed) {
+              const uint64_t qd = ptx::smem_desc_sw128(q_base + off + qoff * 128, 16, 1024);
+              ptx::umma_f16_ss(tmem + (sb ? TM_S1 : TM_S0), kd, qd, idesc_s, kk > 0 ? 1u : 0u);
+            } else {
+              const uint64_t qd = ptx::smem_desc_sw128(q_base + off, 16, 1024);
+              ptx::umma_f16_ss(tmem + (sb ? TM_S1 : TM_S0), qd, kd, idesc_std, kk > 0 ? 1u : 0u);
+            }
           }
           ptx::umma_commit(&ctrl->s_full[sb]);
           ptx::umma_commit(&ctrl->aempty[s]);
         };
-        for (int c = 0; c < nch; ++c) issue_s(c, r0 + c);
+        for (int c = 0; c < nch; ++c) issue_s(c, r0 + c, false);
+        for (int c = 0; c < npre; ++c) issue_s(nch + c, item_k2(c), true);
         bool any = false;
-        if (nch > 0) issue_s(nch, r0 + nch);
         for (int c = 0; c < nch; ++c) {
-          if (c + 1 < nch) issue_s(nch + c + 1, r0 + nch + 2 * (c + 1));
-          const uint32_t vitem = r0 + nch + 2 * c + 1;
+          const uint32_t vitem = item_v2(c);
           const int vs = vitem % NSLOT;
           wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 13);
           wait_bar(ctrl, &ctrl->p_full, (p0 + c) & 1, a.err, 14);
@@ -549,7 +674,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint32_t vbase = slot_base + vs * SLOT_BYTES;
           for (int pi = 0; pi < 2; ++pi) {
             const int pidx = 2 * c + pi;
-            if (pidx >= npages || ctrl->pg_phys[pidx] < 0) continue;
+            if (pidx >= npages || pgp[pidx] < 0) continue;
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const int ks = pi * 4 + k4;   // 16 keys per step
@@ -568,13 +693,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           ptx::umma_commit(&ctrl->aempty[vs]);
           ptx::umma_commit(&ctrl->pv_done);
+          if (c + 2 < nch) issue_s(nch + c + 2, item_k2(c + 2), true);
         }
         ptx::umma_commit(&ctrl->o_done);
       }
-    } else if (warp >= 4) {
-      // ---------------------------------------- softmax warps: one key per thread
-      const int t = tid - 128;                 // key lane in a 128-key chunk, d lane for O^T
-      const int quad = warp - 4;
+    } else {
+      // ---------------------------------------- softmax warps 0-7
+      // TMEM lane t (a q row in pass 1, a key in pass 2, a head dimension
+      // for O^T) is shared by warps `quad` and `quad + 4`, which split the
+      // columns between them (`half`).
+      const int quad = warp & 3;
+      const int half = warp >> 2;
+      const int t = quad * 32 + lane;
       const uint32_t tl = (uint32_t)(quad * 32) << 16;
       // cat: 0 nobody attends the key, 1 every row does, 2 a view row's slot
       auto key_info = [&](int c, int& slot, int& cat, int& xr) {
@@ -582,8 +712,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         cat = 0;
         xr = -1;
         slot = -1;
-        if (pidx >= npages || ctrl->pg_phys[pidx] < 0) return;
-        slot = ctrl->pg_log[pidx] * PS + (t & 63);
+        if (pidx >= npages || pgp[pidx] < 0) return;
+        slot = (int)pgl[pidx] * PS + (t & 63);
         if (slot < L) {
           cat = 1;
           return;
@@ -591,126 +721,177 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int lo = 0, hi = nx - 1;
         while (lo <= hi) {
           const int mid = (lo + hi) >> 1;
-          const int v = ctrl->xs_slot[mid];
+          const int v = xsl[mid];
           if (v == slot) {
             cat = 2;
-            xr = ctrl->xs_row[mid];
+            xr = xsr[mid];
             return;
           }
           if (v < slot) lo = mid + 1; else hi = mid - 1;
         }
       };
-      auto visible = [&](int cat, int xr, int col) -> bool {
-        if (col >= n) return false;
-        if (cat == 1) return true;
-        if (cat == 0) return false;
-        const int rr = ra + col;
-        const int vr = ctrl->row_view[rr];
-        return vr != 0 && vr == ctrl->row_view[xr] && ctrl->row_pos[xr] <= ctrl->row_pos[rr];
+      // Visibility of this thread's key to the 32 rows [32*blk, 32*blk+32)
+      // of the sequence, as a bit mask.
+      auto vis_mask = [&](int cat, int xr, int blk) -> uint32_t {
+        if (cat == 0) return 0u;
+        const int lim = n - 32 * blk;
+        const uint32_t rows = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
+        if (cat == 1) return rows;
+        const int kv = ctrl->row_view[xr], kp = ctrl->row_pos[xr];
+        uint32_t m = 0u;
+        for (int j = 0; j < 32; ++j) {
+          const int col = 32 * blk + j;
+          if (col < n) {
+            const int rr = ra + col;
+            if (ctrl->row_view[rr] == kv && ctrl->row_pos[rr] >= kp) m |= 1u << j;
+          }
+        }
+        return m;
       };
 
-      // ----- pass 1: log-sum-exp of every row
-      for (int c = 0; c < nch; ++c) {
-        int slot, cat, xr;
-        key_info(c, slot, cat, xr);
-        const uint32_t idx = s0 + c;
-        const uint32_t sb = idx & 1;
-        wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 20);
-        ptx::tc_fence_after();
-        const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0);
-        for (int blk = 0; blk < nblk; ++blk) {
-          float v[32];
-          ptx::tmem_ld32(sbase + 32 * blk, v);
-          ptx::tmem_ld_wait();
+      // ----- pass 1: log-sum-exp of every row. S = Q K^T has the group's q
+      // rows on TMEM lanes, so thread t owns q row t; the warp pair of a
+      // quadrant splits the 128 keys of a chunk (half h takes page h), and
+      // the two partial (max, sum) pairs are merged once at the end.
+      {
+        const int r = t - qoff;                    // sequence row of q row t
+        const bool active = r >= 0 && r < n;
+        const bool warp_active = __any_sync(0xffffffffu, active);
+        const int myview = active ? ctrl->row_view[ra + r] : 0;
+        const int mypos = active ? ctrl->row_pos[ra + r] : 0;
+        float m = -INFINITY, l = 0.f;
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t idx = s0 + c;
+          const uint32_t sb = idx & 1;
+          wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 20);
+          ptx::tc_fence_after();
+          if (warp_active) {
+            // keys of this warp's page of the chunk that this row attends:
+            // context slots, then view slots of its own view at positions
+            // <= its own
+            uint64_t km = 0ull;
+            const int pidx = 2 * c + half;
+            if (pidx < npages && pgp[pidx] >= 0) {
+              const int plog = (int)pgl[pidx];
+              const int nv = min(max(L - plog * PS, 0), PS);
+              km = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+              if (nv < PS && myview != 0) {
+                for (int x = 0; x < nx; ++x) {
+                  const int xs = xsl[x];
+                  const int xr = xsr[x];
+                  if (xs / PS == plog && ctrl->row_view[xr] == myview && ctrl->row_pos[xr] <= mypos)
+                    km |= 1ull << (xs % PS);
+                }
+              }
+            }
+            if (!active) km = 0ull;
+            const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + 64 * half;
+#pragma unroll 1
+            for (int blk = 0; blk < 2; ++blk) {
+              float v[32];
+              ptx::tmem_ld32(sbase + 32 * blk, v);
+              const uint32_t mk = blk ? (uint32_t)(km >> 32) : (uint32_t)km;
+              ptx::tmem_ld_wait();
+              // four independent max / sum chains
+              float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            v[j] = visible(cat, xr, 32 * blk + j) ? v[j] * sl2 : -INFINITY;
-          ctrl->red[quad][32 * blk + lane] = reduce_scatter32<true>(v, lane);
-        }
-        named_bar(1, 128);
-        if (t < N16) {
-          const float cm = fmaxf(fmaxf(ctrl->red[0][t], ctrl->red[1][t]),
-                                 fmaxf(ctrl->red[2][t], ctrl->red[3][t]));
-          ctrl->mnew[t] = fmaxf(ctrl->m_run[t], cm);
-        }
-        named_bar(1, 128);
-        for (int blk = 0; blk < nblk; ++blk) {
-          float v[32];
-          ptx::tmem_ld32(sbase + 32 * blk, v);
-          ptx::tmem_ld_wait();
+              for (int j = 0; j < 32; ++j) {
+                v[j] *= sl2;
+                b4[j & 3] = fmaxf(b4[j & 3], ((mk >> j) & 1u) ? v[j] : -INFINITY);
+              }
+              const float mn = fmaxf(m, fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3])));
+              if (mn != -INFINITY) {
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = 32 * blk + j;
-            v[j] = visible(cat, xr, col) ? exp2f(v[j] * sl2 - ctrl->mnew[col]) : 0.f;
+                for (int j = 0; j < 32; ++j) {
+                  const float e = ptx::ex2(v[j] - mn);
+                  s4[j & 3] += ((mk >> j) & 1u) ? e : 0.f;
+                }
+                l = l * ptx::ex2(m - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+                m = mn;
+              }
+            }
           }
-          ctrl->red[quad][32 * blk + lane] = reduce_scatter32<false>(v, lane);
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
         }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
-        named_bar(1, 128);
-        if (t < N16) {
-          const float mn = ctrl->mnew[t];
-          const float sm = ctrl->red[0][t] + ctrl->red[1][t] + ctrl->red[2][t] + ctrl->red[3][t];
-          if (mn != -INFINITY) ctrl->l_run[t] = ctrl->l_run[t] * exp2f(ctrl->m_run[t] - mn) + sm;
-          ctrl->m_run[t] = mn;
+        if (half == 1) {
+          ctrl->pm[t] = m;
+          ctrl->pl[t] = l;
         }
-        named_bar(1, 128);
+        named_bar(1, NSMX);
+        if (half == 0 && active) {
+          const float m1 = ctrl->pm[t], l1 = ctrl->pl[t];
+          const float M = fmaxf(m, m1);
+          const float S = (M == -INFINITY) ? 0.f : l * ptx::ex2(m - M) + l1 * ptx::ex2(m1 - M);
+          ctrl->lse2[r] = S > 0.f ? M + log2f(S) : INFINITY;
+        }
+        named_bar(1, NSMX);
       }
-      if (t < N16)
-        ctrl->lse2[t] = ctrl->l_run[t] > 0.f ? ctrl->m_run[t] + log2f(ctrl->l_run[t]) : INFINITY;
-      // mass row past the context: zero (view slots are written below)
-      if (part)
-        for (int j = L + t; j < plan.row_stride; j += 128) part[j] = 0.f;
-      named_bar(1, 128);
 
-      // ----- pass 2: probabilities, mass, P^T for the P.V product
+      // ----- pass 2: probabilities, mass, P^T for the P.V product. S^T has
+      // the chunk's keys on TMEM lanes (thread t owns key t) and this
+      // sequence's rows on columns; the warp pair splits the rows in
+      // 16-row sub-blocks (sub-block k goes to half k % 2).
+      const int nsub = N16 >> 4;
       for (int c = 0; c < nch; ++c) {
         int slot, cat, xr;
         key_info(c, slot, cat, xr);
         const int pidx = 2 * c + (t >> 6);
-        const bool loaded = pidx < npages && ctrl->pg_phys[pidx] >= 0;
+        const bool loaded = pidx < npages && pgp[pidx] >= 0;
         const uint32_t idx = s0 + nch + c;
         const uint32_t sb = idx & 1;
         wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 21);
         ptx::tc_fence_after();
         const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0);
-        uint32_t ph[4][16], pl[4][16];
-        float mass = 0.f;
+        uint32_t ph[4][8], pq[4][8];
+        float mass2[2] = {0.f, 0.f};
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          if (blk < nblk) {
-            float v[32];
-            ptx::tmem_ld32(sbase + 32 * blk, v);
+        for (int u = 0; u < 4; ++u) {
+          const int k = 2 * u + half;            // 16-row sub-block
+          if (k < nsub) {
+            const uint32_t m16 = (vis_mask(cat, xr, k >> 1) >> (16 * (k & 1))) & 0xffffu;
+            float v[16];
+            ptx::tmem_ld16(sbase + 16 * k, v);
+            const float4* l4 = reinterpret_cast<const float4*>(ctrl->lse2 + 16 * k);
             ptx::tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const int col = 32 * blk + j;
-              const float q0 = visible(cat, xr, col) ? exp2f(v[j] * sl2 - ctrl->lse2[col]) : 0.f;
-              const float q1 =
-                  visible(cat, xr, col + 1) ? exp2f(v[j + 1] * sl2 - ctrl->lse2[col + 1]) : 0.f;
-              mass += q0 + q1;
-              ptx::split_bf16(q0, q1, ph[blk][j >> 1], pl[blk][j >> 1]);
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 ll = l4[j4];
+              const int j = 4 * j4;
+              const float e0 = ptx::ex2(fmaf(v[j], sl2, -ll.x));
+              const float e1 = ptx::ex2(fmaf(v[j + 1], sl2, -ll.y));
+              const float e2 = ptx::ex2(fmaf(v[j + 2], sl2, -ll.z));
+              const float e3 = ptx::ex2(fmaf(v[j + 3], sl2, -ll.w));
+              const float q0 = ((m16 >> j) & 1u) ? e0 : 0.f;
+              const float q1 = ((m16 >> (j + 1)) & 1u) ? e1 : 0.f;
+              const float q2 = ((m16 >> (j + 2)) & 1u) ? e2 : 0.f;
+              const float q3 = ((m16 >> (j + 3)) & 1u) ? e3 : 0.f;
+              mass2[j4 & 1] += (q0 + q1) + (q2 + q3);
+              ptx::split_bf16(q0, q1, ph[u][j >> 1], pq[u][j >> 1]);
+              ptx::split_bf16(q2, q3, ph[u][(j >> 1) + 1], pq[u][(j >> 1) + 1]);
             }
           }
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
-        if (part && cat != 0) part[slot] = mass;
+        // both halves add into the zeroed mass row; two addends, so the
+        // result does not depend on their order
+        if (part && cat != 0 && nsub > half) atomicAdd(part + slot, mass2[0] + mass2[1]);
         // V rows of keys nobody attends may hold anything (page tails):
-        // zero them so that 0 * V stays 0 in the P.V product.
-        const uint32_t vitem = r0 + nch + 2 * c + 1;
+        // zero them so that 0 * V stays 0 in the P.V product (each half
+        // clears one 64-dimension half of the row).
+        const uint32_t vitem = item_v2(c);
         const int vs = vitem % NSLOT;
         if (loaded && cat == 0) {
           wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 22);
-          uint8_t* vrow = smem + SLOT_OFF + vs * SLOT_BYTES + (t >> 6) * BOX_BYTES + (t & 63) * 128;
+          uint8_t* vrow = smem + SLOT_OFF + vs * SLOT_BYTES + half * HALF_BYTES +
+                          (t >> 6) * BOX_BYTES + (t & 63) * 128;
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
-            *reinterpret_cast<uint4*>(vrow + HALF_BYTES + ch * 16) = z;
-          }
+          for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
         }
         // The P^T buffers are free once the previous P.V product completed.
         const uint32_t pidx_g = p0 + c;
@@ -718,19 +899,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* pth = smem + PT_OFF;
         uint8_t* ptl = pth + PT_BYTES;
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-          if (blk < nblk) {
+        for (int u = 0; u < 4; ++u) {
+          const int k = 2 * u + half;
+          if (k < nsub) {
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              const int nb = 4 * blk + g8;     // 8-row block of the sequence
-              if (8 * nb < N16) {
-                *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) =
-                    make_uint4(ph[blk][4 * g8], ph[blk][4 * g8 + 1], ph[blk][4 * g8 + 2],
-                               ph[blk][4 * g8 + 3]);
-                *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) =
-                    make_uint4(pl[blk][4 * g8], pl[blk][4 * g8 + 1], pl[blk][4 * g8 + 2],
-                               pl[blk][4 * g8 + 3]);
-              }
+            for (int g8 = 0; g8 < 2; ++g8) {
+              const int nb = 2 * k + g8;     // 8-row block of the sequence
+              *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) =
+                  make_uint4(ph[u][4 * g8], ph[u][4 * g8 + 1], ph[u][4 * g8 + 2], ph[u][4 * g8 + 3]);
+              *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) =
+                  make_uint4(pq[u][4 * g8], pq[u][4 * g8 + 1], pq[u][4 * g8 + 2], pq[u][4 * g8 + 3]);
             }
           }
         }
@@ -738,17 +916,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctrl->p_full);
       }
-      // ----- O^T -> out (thread t = head dimension t)
+      // ----- O^T -> out (thread t = head dimension t; the halves split rows)
       wait_bar(ctrl, &ctrl->o_done, ocount & 1, a.err, 24);
       ptx::tc_fence_after();
-      for (int blk = 0; blk < nblk; ++blk) {
-        float v[32];
-        ptx::tmem_ld32(tmem + tl + TM_O + 32 * blk, v);
+      for (int k = half; k < nsub; k += 2) {
+        float v[16];
+        ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int r = 32 * blk + j;
-          if (r < n) a.out[(size_t)(row0 + ra + r) * H + h * D + t] = any_page ? v[j] : 0.f;
+        for (int j = 0; j < 16; ++j) {
+          const int rr = 16 * k + j;
+          if (rr < n) a.out[(size_t)(gr0 + rr) * H + h * D + t] = any_page ? v[j] : 0.f;
         }
       }
       ptx::tc_fence_before();
@@ -757,17 +935,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     scount = s0 + 2 * nch;
     pcount = p0 + nch;
     ++ocount;
-    __syncwarp();
-    __syncthreads();
   }
 
   // ================================================================ teardown
-  if (warp == 1 && lane == 0) {
+  if (warp == kMmaWarp && lane == 0) {
     // every tcgen05 operation issued by this thread has completed
     ptx::umma_commit(&ctrl->mma_done);
     ptx::mbar_wait(&ctrl->mma_done, 1, WAIT_NS);
   }
-  if (warp == 0 && lane == 0 && ring > 0) {
+  if (warp == kProducerWarp && lane == 0 && ring > 0) {
     // the last chunk loads have landed (they have, unless a wait timed out)
     for (uint32_t it = ring > NSLOT ? ring - NSLOT : 0; it < ring; ++it)
       ptx::mbar_wait(&ctrl->afull[it % NSLOT], (it / NSLOT) & 1, WAIT_NS);
@@ -775,14 +951,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) ptx::tmem_dealloc(tmem, TMEM_COLS);
+  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace
 
 size_t step_bf16_smem_bytes() { return SMEM_BYTES; }
 
-cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* tmap_x,
+cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* const* tmap_x,
                              const void* tmap_w, const void* tmap_k, const void* tmap_v,
                              cudaStream_t stream) {
   static bool attr_set = false;
@@ -795,7 +971,9 @@ cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void
   const int grid = plan.n_groups * a.n_heads;
   if (grid == 0) return cudaSuccess;
   step_bf16_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
-      plan, a, *reinterpret_cast<const CUtensorMap*>(tmap_x),
+      plan, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
+      *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
+      *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
       *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_k),
       *reinterpret_cast<const CUtensorMap*>(tmap_v));
   return cudaGetLastError();
