@@ -53,6 +53,30 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def captured_traffic(name: str):
+    """DRAM bytes per launch of the step kernel from the committed ncu
+    summary for this workload, if the kernel sources are unchanged since the
+    capture (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"step_bf16_{name}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    want = None
+    traffic = None
+    for line in txt.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1])
+        if line.startswith("kernel_sources_sha256:"):
+            want = line.split(":", 1)[1].split()
+    if traffic is None or want is None:
+        return None
+    csrc = os.path.join(ROOT, "kv_cache_attention_flash_b200", "csrc")
+    have = [hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()
+            for f in ("step_bf16.cu", "ptx.cuh")]
+    return traffic if have == want else None
+
+
 def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
         int(os.environ.get("LOCAL_RANK", "0"))
@@ -394,8 +418,9 @@ def run_native(args):
         achieved, peak, unit = fl / kern_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     else:
         achieved, peak, unit = byt / kern_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    traffic = args.traffic if args.traffic is not None else captured_traffic(spec.name)
     roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-            "traffic": args.traffic, "peak_source": f"{peak_src} (burst)",
+            "traffic": traffic, "peak_source": f"{peak_src} (burst)",
             "kernel": "fdllm_layer_step (fused step kernel + mass reduce), layer 0",
             "kernel_us": kern_s * 1e6, "algorithmic_bytes": byt, "algorithmic_flops": fl,
             "hbm_gbs_achieved": byt / kern_s / 1e9,
