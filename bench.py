@@ -57,7 +57,6 @@ def captured_traffic(name: str):
     """DRAM bytes per launch of the step kernel from the committed ncu
     summary for this workload, if the kernel sources are unchanged since the
     capture (else None)."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", f"step_bf16_{name}.md")
     if not os.path.exists(path):
         return None
@@ -72,9 +71,20 @@ def captured_traffic(name: str):
     if traffic is None or want is None:
         return None
     csrc = os.path.join(ROOT, "kv_cache_attention_flash_b200", "csrc")
-    have = [hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()
-            for f in ("step_bf16.cu", "ptx.cuh")]
+    have = [code_hash(os.path.join(csrc, f)) for f in ("step_bf16.cu", "ptx.cuh")]
     return traffic if have == want else None
+
+
+def code_hash(path: str) -> str:
+    """sha256 of a CUDA source with // comments and blank lines removed, so
+    that an edit of comments alone keeps a capture valid."""
+    import hashlib
+    lines = []
+    for line in open(path).read().splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code.strip():
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
 
 
 def dist_env():
@@ -99,6 +109,14 @@ def reduce_sum(value: float, device) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def aggregate(total_ms_local: float, units_local: float, device):
+    """Whole-job throughput of independent replicas: the slowest rank's time
+    and the units of all ranks. Returns (max ms, total units, units/s)."""
+    total_ms = reduce_max(total_ms_local, device)
+    units_all = reduce_sum(units_local, device)
+    return total_ms, units_all, units_all / (total_ms / 1000.0)
 
 
 def barrier():
@@ -403,10 +421,7 @@ def run_native(args):
     step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
     layer_ms = [ev_ls[i].elapsed_time(ev_le[i]) for i in range(args.steps)]
     total_ms_local = float(sum(step_ms))
-    total_ms = reduce_max(total_ms_local, dev)
-    rows_local = meta.total_rows * args.steps
-    rows_all = reduce_sum(rows_local, dev)
-    value = rows_all / (total_ms / 1000.0)
+    total_ms, _, value = aggregate(total_ms_local, meta.total_rows * args.steps, dev)
 
     # roofline of the dominant kernel (the fused layer step, layer 0)
     byt, fl = W.algorithmic_bytes_flops(spec, meta)

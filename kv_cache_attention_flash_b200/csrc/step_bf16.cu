@@ -17,17 +17,20 @@
 //   rotate-half RoPE to q and k, round to bf16, keep q in shared memory in
 //   the UMMA operand layout, and copy k/v rows to their cache slots with
 //   coalesced 16-byte stores.
-// Phase 3 (attention), per sequence of the group, on the tensor cores in
-//   transposed form so that a sequence of only 16..128 rows wastes no MMA
-//   rows: S^T = K Q^T (keys on TMEM lanes, the sequence's rows on columns)
-//   and O^T += V^T P^T. K and V pages are gathered by TMA through the block
-//   table, two 64-slot pages per 128-key chunk, into a 3-slot ring.
-//   Pass 1 finds every row's log-sum-exp (column max/sum across the 128
-//   key lanes by a shuffle reduce-scatter); pass 2 forms the exact
-//   probabilities, whose per-key sums over the rows are the attention mass
-//   (one thread per key, no cross-thread reduction), and feeds P^T to the
-//   P.V product as bf16 hi + lo parts. The Flash-Verify two-view rule
-//   (paragraph 3 of the same page) decides visibility of fresh view keys.
+// Phase 3 (attention), per sequence of the group, on the tensor cores. K
+//   and V pages are gathered by TMA through the block table, two 64-slot
+//   pages per 128-key chunk, into a 3-slot ring.
+//   Pass 1 finds every row's log-sum-exp from S = Q K^T (the group's q rows
+//   on TMEM lanes, so each thread keeps its own row's running max and sum;
+//   the two warps of a lane quadrant take one page of the chunk each and
+//   merge once at the end).
+//   Pass 2 runs in transposed form so that a sequence of only 16..128 rows
+//   wastes no MMA rows: S^T = K Q^T (keys on lanes, the sequence's rows on
+//   columns) gives the exact probabilities, whose per-key sums over the
+//   rows are the attention mass (one thread per key, no cross-thread
+//   reduction), and O^T += V^T P^T takes P^T as bf16 hi + lo parts. The
+//   Flash-Verify two-view rule (paragraph 3 of the same page) decides
+//   visibility of fresh view keys.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
