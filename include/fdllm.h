@@ -180,6 +180,44 @@ FDLLM_API fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_
                                   int32_t row_stride, int32_t k, const int32_t* exclude_cu,
                                   const int32_t* exclude_slots, int32_t* tracked, void* stream);
 
+/* The layer step of fdllm_layer_step without a handle and without any
+ * device allocation. The paper has no counterpart: it exists for callers
+ * that cannot call cudaMalloc when they run a step, such as a serving
+ * engine that has already given nearly all free HBM to its KV pool, or a
+ * framework whose own allocator must account for every device byte.
+ *   cfg, k_pool, v_pool: as for fdllm_cache_create (same rules).
+ *   rope_cos, rope_sin: DEVICE fp32 [cfg->max_position][cfg->head_dim / 2],
+ *     16-byte aligned, owned by the caller: entry [p][i] is the cosine / sine
+ *     of p * rope_theta^(-2i/head_dim), rounded to fp32 (the tables that
+ *     fdllm_cache_create computes in double).
+ *   layer, step, x, wqkv, positions, block_table, view_mask, out, attn_mass,
+ *     stream: as for fdllm_layer_step; cfg->max_batch and
+ *     cfg->max_slots_per_seq bound the step the same way.
+ * Scratch: the per-head attention-mass partials and the device error word
+ * live in one fixed 8 MiB array in the library's device image, which every
+ * GPU that loads the library holds until the process exits. With attn_mass
+ * non-NULL, n_heads * batch * max_blocks_per_seq * page_size must be at most
+ * 2,097,088 floats, else FDLLM_ERR_UNSUPPORTED (nothing enqueued).
+ * The first call on each device looks up the array's device address and
+ * clears its error word, synchronising `stream` once; make that first call
+ * before any stream capture. Later calls enqueue work only (no host sync
+ * unless step->validate is 1).
+ * Every call on a device shares the array, so calls whose work overlaps on
+ * the GPU (other streams, other threads) race on it and give wrong mass or
+ * error reports; serialise them. The partial rows a call uses are zeroed by
+ * its own kernel, so contents left by an earlier call do not matter.
+ * Errors: device-detected errors are kept in the shared error word and
+ * reported, then cleared, by the next call with step->validate = 1
+ * (FDLLM_ERR_DEVICE_BOUNDS or FDLLM_ERR_TIMEOUT); fdllm_check does not see
+ * them. No cudaMalloc, cudaFree or other device allocation happens; host
+ * planning uses ordinary host memory as in fdllm_layer_step. */
+FDLLM_API fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_pool,
+                                      void* v_pool, const float* rope_cos, const float* rope_sin,
+                                      int32_t layer, const fdllm_step* step, const void* x,
+                                      const void* wqkv, const int32_t* positions,
+                                      const int32_t* block_table, const int8_t* view_mask,
+                                      float* out, float* attn_mass, void* stream);
+
 /* Synchronises `stream`, reads and clears the handle's device error word.
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
  * FDLLM_ERR_CUDA. */
@@ -191,8 +229,9 @@ FDLLM_API const char* fdllm_status_string(fdllm_status status);
 /* Message for the last failing call on this thread ("" if none). */
 FDLLM_API const char* fdllm_last_error(void);
 
-/* Number of kernel launches the last successful fdllm_layer_step or
- * fdllm_select_tracked call on this thread enqueued. */
+/* Number of kernel launches the last successful fdllm_layer_step,
+ * fdllm_layer_step_noalloc or fdllm_select_tracked call on this thread
+ * enqueued. */
 FDLLM_API int32_t fdllm_last_launch_count(void);
 
 #ifdef __cplusplus

@@ -24,7 +24,8 @@ from ._lib import (FDLLM_BF16, FDLLM_F32, FDLLM_OK, CacheConfig, FdllmError, Ste
                    check_status, load)
 
 __all__ = [
-    "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_select_tracked",
+    "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_layer_step_noalloc",
+    "fdllm_select_tracked",
     "fdllm_check", "fdllm_last_launch_count", "FlashCache", "FdllmError", "load",
 ]
 
@@ -97,6 +98,47 @@ def fdllm_layer_step(handle: int, layer: int, cu_rows: Sequence[int], seq_lens: 
               _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0)
     check_status(lib.fdllm_layer_step(
         handle, int(layer), ctypes.byref(st), _dev_ptr(x, None, "x"), _dev_ptr(wqkv, None, "wqkv"),
+        _dev_ptr(positions, torch.int32, "positions"), _dev_ptr(block_table, torch.int32, "block_table"),
+        _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, torch.float32, "out"),
+        _dev_ptr(attn_mass, torch.float32, "attn_mass"), _stream_ptr(stream)))
+
+
+def fdllm_layer_step_noalloc(n_layers: int, n_heads: int, head_dim: int, page_size: int,
+                             num_pages: int, max_position: int, rope_theta: float, dtype: str,
+                             max_batch: int, max_slots_per_seq: int, k_pool: torch.Tensor,
+                             v_pool: torch.Tensor, rope_cos: torch.Tensor, rope_sin: torch.Tensor,
+                             layer: int, cu_rows: Sequence[int], seq_lens: Sequence[int],
+                             max_blocks_per_seq: int, x: torch.Tensor, wqkv: torch.Tensor,
+                             positions: torch.Tensor, block_table: torch.Tensor,
+                             view_mask: Optional[torch.Tensor], out: torch.Tensor,
+                             attn_mass: Optional[torch.Tensor],
+                             slots: Optional[torch.Tensor] = None, validate: bool = False,
+                             stream=None) -> None:
+    """The layer step without a handle or any device allocation, for callers
+    that cannot call cudaMalloc when they step (their HBM is already handed
+    to a KV pool or to their own allocator). The library keeps its scratch
+    in a fixed per-device array; overlapping calls on one GPU race on it.
+    rope_cos / rope_sin: caller-owned fp32 [max_position][head_dim / 2]
+    tables (see include/fdllm.h)."""
+    lib = load()
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    cfg = CacheConfig(n_layers, n_heads, head_dim, page_size, num_pages, max_position, max_batch,
+                      max_slots_per_seq, float(rope_theta),
+                      FDLLM_BF16 if dtype == "bf16" else FDLLM_F32)
+    half = head_dim // 2
+    for nm, t in (("rope_cos", rope_cos), ("rope_sin", rope_sin)):
+        if tuple(t.shape) != (max_position, half):
+            raise ValueError(f"{nm} must have shape {(max_position, half)}, got {tuple(t.shape)}")
+    cu = _host_i32(cu_rows)
+    sl = _host_i32(seq_lens)
+    st = Step(len(sl), int(cu[-1]), int(max_blocks_per_seq),
+              cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+              sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+              _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0)
+    check_status(lib.fdllm_layer_step_noalloc(
+        ctypes.byref(cfg), _dev_ptr(k_pool, tdt, "k_pool"), _dev_ptr(v_pool, tdt, "v_pool"),
+        _dev_ptr(rope_cos, torch.float32, "rope_cos"), _dev_ptr(rope_sin, torch.float32, "rope_sin"),
+        int(layer), ctypes.byref(st), _dev_ptr(x, None, "x"), _dev_ptr(wqkv, None, "wqkv"),
         _dev_ptr(positions, torch.int32, "positions"), _dev_ptr(block_table, torch.int32, "block_table"),
         _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, torch.float32, "out"),
         _dev_ptr(attn_mass, torch.float32, "attn_mass"), _stream_ptr(stream)))

@@ -44,6 +44,9 @@ SIGNATURES = {
     "fdllm_cache_create": (_i32, [ctypes.POINTER(CacheConfig), _vp, _vp, _vp, ctypes.POINTER(_vp)]),
     "fdllm_cache_destroy": (None, [_vp]),
     "fdllm_layer_step": (_i32, [_vp, _i32, ctypes.POINTER(Step), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fdllm_layer_step_noalloc": (_i32, [ctypes.POINTER(CacheConfig), _vp, _vp, _vp, _vp, _i32,
+                                        ctypes.POINTER(Step), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _vp]),
     "fdllm_select_tracked": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fdllm_check": (_i32, [_vp, _vp]),
     "fdllm_status_string": (ctypes.c_char_p, [_i32]),

@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <mutex>
 #include <set>
 #include <string>
 #include <vector>
@@ -484,6 +485,165 @@ fdllm_status fdllm_check(fdllm_cache* h, void* stream) {
   if (code == kDevTimeout)
     return fail(FDLLM_ERR_TIMEOUT, "device: %s (site %d)", what[code], w[1]);
   return fail(FDLLM_ERR_DEVICE_BOUNDS, "device: %s (detail %d)", what[code], w[1]);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Layer step that allocates no device memory.
+//
+// Some callers cannot call cudaMalloc at the time they run a step: a serving
+// engine that has already handed nearly all free HBM to its paged KV pool
+// (a late cudaMalloc would fail or fragment that reservation), or a host
+// framework whose own allocator must account for every device byte. For
+// them the step's only scratch, the per-head attention-mass partial sums
+// and the device error word, lives in the fixed array below, part of the
+// library's device image, instead of in a handle's cudaMalloc'd workspace.
+// The caller passes the pools and the RoPE tables it owns; nothing else is
+// needed, so no handle is created.
+//
+// Layout of the array: bytes [0, 16) the error word (int32[4]; must start at
+// zero: cleared on the first call on each device and after every report),
+// bytes [256, end) the mass partials [n_heads][batch][max_blocks*page_size]
+// fp32 (each row the step uses is zeroed by the kernel before it
+// accumulates, so stale contents from an earlier call do not matter).
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB per device
+constexpr size_t kNoAllocPartOffset = 256;
+constexpr size_t kNoAllocPartFloats = (kNoAllocScratchBytes - kNoAllocPartOffset) / sizeof(float);
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices];   // device address of the array, per device
+
+// Device address of g_noalloc_scratch on the current device. The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current),
+// zeroes the error word on `stream` and waits for that; later calls reuse
+// the address.
+fdllm_status noalloc_scratch(cudaStream_t stream, void** addr) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "layer_step_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step_noalloc: device ordinal %d >= %d", dev,
+                kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess)
+      return cuda_fail(e, "layer_step_noalloc: cudaGetSymbolAddress");
+    if ((e = cudaMemsetAsync(p, 0, 4 * sizeof(int), stream)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(stream)) != cudaSuccess)
+      return cuda_fail(e, "layer_step_noalloc: clear error word");
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return FDLLM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_pool, void* v_pool,
+                                      const float* rope_cos, const float* rope_sin, int32_t layer,
+                                      const fdllm_step* st, const void* x, const void* wqkv,
+                                      const int32_t* positions, const int32_t* block_table,
+                                      const int8_t* view_mask, float* out, float* attn_mass,
+                                      void* stream) {
+  if (!cfg || !st) return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: null cfg or step");
+  if (!k_pool || !v_pool || !rope_cos || !rope_sin)
+    return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: null pool or RoPE table");
+  if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool) |
+       reinterpret_cast<uintptr_t>(rope_cos) | reinterpret_cast<uintptr_t>(rope_sin)) & 15)
+    return fail(FDLLM_ERR_INVALID_ARG,
+                "layer_step_noalloc: pools and RoPE tables must be 16-byte aligned");
+  // The same configuration rules as fdllm_cache_create.
+  const fdllm_cache_config& c = *cfg;
+  if (c.n_layers <= 0 || c.n_heads <= 0 || c.head_dim <= 0 || c.page_size <= 0 ||
+      c.num_pages <= 0 || c.max_position <= 0 || c.max_batch <= 0 || c.max_slots_per_seq <= 0)
+    return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: sizes must be positive");
+  if (c.dtype != FDLLM_BF16 && c.dtype != FDLLM_F32)
+    return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: unknown dtype %d", c.dtype);
+  if (c.head_dim % 2)
+    return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: head_dim must be even (RoPE pairs)");
+  if (c.dtype == FDLLM_BF16 && c.head_dim != 128)
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step_noalloc: bf16 kernels serve head_dim 128 only");
+  if (c.dtype == FDLLM_F32 && (c.head_dim > 128 || c.head_dim % 32))
+    return fail(FDLLM_ERR_UNSUPPORTED,
+                "layer_step_noalloc: fp32 kernel serves head_dim 32/64/96/128");
+  if (c.max_batch > kMaxBatch)
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step_noalloc: max_batch > %d", kMaxBatch);
+  if (c.dtype == FDLLM_BF16 && c.page_size != kBf16PageSize)
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step_noalloc: bf16 kernels gather %d-slot pages",
+                kBf16PageSize);
+  if ((long long)c.n_layers * c.num_pages * c.n_heads * c.page_size >= (1ll << 31))
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step_noalloc: pool has 2^31 or more slot rows");
+  if (st->batch <= 0 || st->max_blocks_per_seq <= 0)
+    return fail(FDLLM_ERR_INVALID_ARG,
+                "layer_step_noalloc: batch and max_blocks_per_seq must be positive");
+  // The fixed scratch bounds the mass partials: n_heads * batch * row length.
+  if (attn_mass) {
+    const long long need =
+        (long long)c.n_heads * st->batch * st->max_blocks_per_seq * c.page_size;
+    if (need > (long long)kNoAllocPartFloats)
+      return fail(FDLLM_ERR_UNSUPPORTED,
+                  "layer_step_noalloc: the attention-mass scratch needs %lld floats "
+                  "(n_heads * batch * max_blocks_per_seq * page_size), more than the %zu that "
+                  "fit in the library's fixed %zu-byte buffer; pass attn_mass = NULL or use "
+                  "fdllm_layer_step",
+                  need, kNoAllocPartFloats, kNoAllocScratchBytes);
+  }
+
+  void* scratch = nullptr;
+  fdllm_status ss = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &scratch);
+  if (ss != FDLLM_OK) return ss;
+
+  // A handle on the stack over the caller's memory and the fixed scratch;
+  // fdllm_layer_step does the rest (checks, plan, launches).
+  fdllm_cache h;
+  memset(&h, 0, sizeof(h));
+  h.cfg = c;
+  h.k_pool = k_pool;
+  h.v_pool = v_pool;
+  if (c.dtype == FDLLM_BF16) {
+    const uint64_t rows = (uint64_t)c.n_layers * c.num_pages * c.n_heads * c.page_size;
+    if (!encode_bf16_2d(&h.tmap_k, k_pool, rows, (uint64_t)c.head_dim, (uint32_t)c.page_size) ||
+        !encode_bf16_2d(&h.tmap_v, v_pool, rows, (uint64_t)c.head_dim, (uint32_t)c.page_size))
+      return fail(FDLLM_ERR_CUDA, "layer_step_noalloc: cuTensorMapEncodeTiled failed for the pools");
+  }
+  cudaGetDevice(&h.device);
+  h.rope_cos = const_cast<float*>(rope_cos);
+  h.rope_sin = const_cast<float*>(rope_sin);
+  h.mass_part = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocPartOffset);
+  h.mass_part_floats = kNoAllocPartFloats;
+  h.err = static_cast<int*>(scratch);
+
+  fdllm_status s = fdllm_layer_step(&h, layer, st, x, wqkv, positions, block_table, view_mask, out,
+                                    attn_mass, stream);
+  if (s != FDLLM_OK || !st->validate) return s;
+  // validate = 1: fdllm_layer_step has synchronised the stream; report and
+  // clear what the kernels recorded in the error word.
+  int w[4];
+  cudaError_t e;
+  if ((e = cudaMemcpy(w, h.err, sizeof(w), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "layer_step_noalloc: read error word");
+  if (w[0] == 0) return FDLLM_OK;
+  if ((e = cudaMemsetAsync(h.err, 0, sizeof(w), reinterpret_cast<cudaStream_t>(stream))) !=
+      cudaSuccess)
+    return cuda_fail(e, "layer_step_noalloc: clear error word");
+  if (w[0] == kDevTimeout)
+    return fail(FDLLM_ERR_TIMEOUT, "device: bounded wait timed out (site %d)", w[1]);
+  return fail(FDLLM_ERR_DEVICE_BOUNDS, "device: metadata out of range (code %d, detail %d)", w[0],
+              w[1]);
 }
 
 }  // extern "C"
