@@ -340,8 +340,11 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   // multiple of 16 q rows (the attention MMA's N granularity), packed first
   // fit in order of decreasing size. The bf16 kernel also keeps a group's
   // attended page list on chip (at most kBf16GroupPages entries, bounded by
-  // context pages + rows). Groups are then ordered by decreasing attention
-  // work so that the costliest tiles start first.
+  // context pages + rows) and serves at most 8 sequences per group. Groups
+  // are launched in order of decreasing attention work, head by head within
+  // a group, so that the longest tiles start first and the short ones fill
+  // in at the end. Work is counted in 128-key chunks (a chunk costs about
+  // the same whatever the row count) plus one chunk per sequence.
   {
     struct Grp {
       int pad, pages;
@@ -353,13 +356,19 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
       plan.seq_qoff[b] = 0;
       if (st->cu_rows[b + 1] > st->cu_rows[b]) idx.push_back(b);
     }
-    auto n16 = [&](int b) { return (st->cu_rows[b + 1] - st->cu_rows[b] + 15) & ~15; };
+    auto rows_of = [&](int b) { return st->cu_rows[b + 1] - st->cu_rows[b]; };
+    auto n16 = [&](int b) { return (rows_of(b) + 15) & ~15; };
     auto pages = [&](int b) {
-      return (st->seq_lens[b] + c.page_size - 1) / c.page_size + st->cu_rows[b + 1] - st->cu_rows[b];
+      return (st->seq_lens[b] + c.page_size - 1) / c.page_size + rows_of(b);
+    };
+    auto work = [&](int b) -> long long {
+      const int ctx = (st->seq_lens[b] + c.page_size - 1) / c.page_size;
+      const int extra = (rows_of(b) + c.page_size - 1) / c.page_size + 1;
+      return (ctx + extra + 1) / 2 + 1;
     };
     std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
       if (n16(x) != n16(y)) return n16(x) > n16(y);
-      return st->seq_lens[x] > st->seq_lens[y];
+      return work(x) > work(y);
     });
     std::vector<Grp> groups;
     for (int b : idx) {
@@ -374,10 +383,9 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
         groups.push_back(Grp{0, 0, 0, {}});
         dst = &groups.back();
       }
-      plan.seq_qoff[b] = dst->pad;
       dst->pad += n16(b);
       dst->pages += pages(b);
-      dst->cost += (long long)(st->seq_lens[b] + c.page_size) * n16(b);
+      dst->cost += work(b);
       dst->seqs.push_back(b);
     }
     if ((int)groups.size() > kMaxGroups)
@@ -387,7 +395,12 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
     int k = 0;
     for (size_t gi = 0; gi < groups.size(); ++gi) {
       plan.group_seq0[gi] = k;
-      for (int b : groups[gi].seqs) plan.seq_order[k++] = b;
+      int off = 0;
+      for (int b : groups[gi].seqs) {
+        plan.seq_order[k++] = b;
+        plan.seq_qoff[b] = off;
+        off += n16(b);
+      }
     }
     plan.group_seq0[groups.size()] = k;
     plan.n_groups = (int)groups.size();

@@ -12,7 +12,8 @@
 // Phase 1 (projection): [128 rows x H] x [H x 384], the 384 columns being
 //   this head's q | k | v blocks of Wqkv. TMA streams x and Wqkv tiles
 //   (128-byte swizzle) through a 3-stage mbarrier pipeline; one thread
-//   issues tcgen05.mma (M=128, N=128, K=16, bf16 -> fp32) into TMEM.
+//   issues tcgen05.mma (M=128, N=256 for q|k and N=128 for v, K=16,
+//   bf16 -> fp32) into TMEM.
 // Phase 2 (epilogue): all 8 warps read the accumulator from TMEM, apply
 //   rotate-half RoPE to q and k, round to bf16, keep q in shared memory in
 //   the UMMA operand layout, and copy k/v rows to their cache slots with
@@ -231,8 +232,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int h = blockIdx.x / plan.n_groups;
-  const int g = blockIdx.x % plan.n_groups;
+  // tiles are numbered group-major (groups in order of decreasing work)
+  const int g = blockIdx.x / a.n_heads;
+  const int h = blockIdx.x % a.n_heads;
   // sequences of this group: plan.seq_order[seq_a .. seq_b); sequence b
   // owns q rows [seq_qoff[b], seq_qoff[b] + n_b) of the 128-row tile, which
   // are also the TMEM lanes of the projection
@@ -326,6 +328,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {   // MMA issuer
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, 128, false, true);
+      constexpr uint32_t idesc256 = ptx::idesc_bf16_f32(BM, 256, false, true);
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % STAGES;
         const int u = kb / STAGES;
@@ -337,14 +340,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int kk = 0; kk < BK / 16; ++kk) {
           // A: K-major rows of 128 bytes; 8-row atoms 1024 bytes apart.
           const uint64_t ad = ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024);
-#pragma unroll
-          for (int blk = 0; blk < 3; ++blk) {
-            // B: N-major (Wqkv rows are K); 64-column boxes 8 KB apart,
-            // 8-row K groups 1024 bytes apart; K16 slice = 16 rows = 2 KB.
-            const uint64_t bd = ptx::smem_desc_sw128(b_base + blk * 2 * BOX_BYTES + kk * 2048,
-                                                     BOX_BYTES, 1024);
-            ptx::umma_f16_ss(tmem + blk * 128, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          // B: N-major (Wqkv rows are K); 64-column boxes 8 KB apart, 8-row
+          // K groups 1024 bytes apart; K16 slice = 16 rows = 2 KB. q and k
+          // (four boxes, 256 columns) go in one N=256 product, which reads
+          // the A tile from shared memory once for both; v is N=128.
+          const uint64_t bqk = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
+          ptx::umma_f16_ss(tmem, ad, bqk, idesc256, (kb | kk) != 0 ? 1u : 0u);
+          const uint64_t bv = ptx::smem_desc_sw128(b_base + 4 * BOX_BYTES + kk * 2048,
+                                                   BOX_BYTES, 1024);
+          ptx::umma_f16_ss(tmem + 256, ad, bv, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         ptx::umma_commit(&ctrl->empty[s]);
       }

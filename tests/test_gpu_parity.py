@@ -45,6 +45,51 @@ def test_parity_full_size(name):
     check_dense(spec, meta, x, w, kp, vp, g)
 
 
+def test_parity_stacked32_sampled_layers():
+    """The 32-layer stack at full size (batch 4, 8192 cached slots per
+    sequence, 32 window + 64 tracked rows): every layer runs on the GPU in
+    stream order through one handle over the full pools, as the benchmark
+    runs them; three sampled layers are checked against the oracle. One-hot
+    x rows make each projection exact, so the plain bound applies."""
+    from gpu_case import GpuRun
+    spec = W.get_spec("stacked32_b4")
+    sh = spec.shape
+    meta = W.make_meta(spec, 0)
+    dev = "cuda"
+    nl = sh.n_layers
+    sampled = (0, 13, nl - 1)
+    kp, vp = W.make_pools(spec, meta, 0, device=dev)
+    pre = {l: (W.bits_np(kp[l:l + 1]), W.bits_np(vp[l:l + 1])) for l in sampled}
+    xs = [W.make_x_onehot(spec, meta, 100 + l, device=dev) for l in range(nl)]
+    ws = [W.make_w(spec, 0, layer=l, device=dev) for l in range(nl)]
+    ps = sh.page_size
+    cache = fd.FlashCache(nl, sh.n_heads, sh.head_dim, ps, meta.num_pages, meta.max_position,
+                          sh.rope_theta, sh.dtype, max_batch=meta.batch,
+                          max_slots_per_seq=meta.max_blocks * ps, k_pool=kp, v_pool=vp)
+    pos = torch.from_numpy(meta.positions).to(dev)
+    slots = torch.from_numpy(meta.slots).to(dev)
+    bt = torch.from_numpy(meta.block_table).to(dev)
+    outs, masses = {}, {}
+    for l in range(nl):
+        out, mass = cache.step(l, meta.cu_rows, meta.seq_lens, xs[l], ws[l], pos, bt, slots=slots)
+        if l in sampled:
+            outs[l], masses[l] = out, mass
+    cache.check()
+    sl = torch.from_numpy(meta.seq_lens).to(dev)
+    ecu = torch.from_numpy(meta.exclude_cu).to(dev)
+    ex = meta.exclude_slots if len(meta.exclude_slots) else np.zeros(1, np.int32)
+    esl = torch.from_numpy(ex).to(dev)
+    for l in sampled:
+        tracked = fd.fdllm_select_tracked(masses[l], sl, meta.track_k, ecu, esl).cpu().numpy()
+        g = GpuRun(outs[l].cpu().numpy(), masses[l].cpu().numpy(), tracked,
+                   W.bits_np(cache.k_pool[l]), W.bits_np(cache.v_pool[l]))
+        kb, vb = pre[l]
+        o = O.layer_step(sh, kb, vb, 0, W.bits_np(xs[l]), W.bits_np(ws[l]), meta.positions,
+                         meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table, meta.view)
+        compare(spec, meta, g, o, kb, vb, mode="exact")
+    cache.close()
+
+
 @pytest.mark.parametrize("name", ["small_bf16_divergent", "small_bf16_two_view", "llada8b_b1",
                                   "b32_divergent", "two_view_b8"])
 def test_parity_exact_projection_plain_tolerance(name):
