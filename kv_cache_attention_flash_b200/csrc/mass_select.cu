@@ -30,6 +30,43 @@ __global__ void mass_reduce_kernel(const __grid_constant__ StepPlan plan, const 
   mass[(size_t)b * plan.row_stride + j] = s;
 }
 
+// The same reduction four slots per thread, for row strides that are a
+// multiple of 4 and a 16-byte aligned output; heads are summed in the same
+// order, so both give the same bits.
+__global__ void mass_reduce4_kernel(const __grid_constant__ StepPlan plan, const float* part,
+                                    float* mass, int n_heads) {
+  const int b = blockIdx.y;
+  const int j = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (j >= plan.row_stride) return;
+  const int n = plan.cu_rows[b + 1] - plan.cu_rows[b];
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (n > 0) {
+    const size_t hs = (size_t)plan.batch * plan.row_stride;
+    const float* p = part + (size_t)b * plan.row_stride + j;
+    // 16 heads' loads in flight at a time, added in head order
+    for (int h0 = 0; h0 < n_heads; h0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (h0 + u < n_heads) v[u] = __ldg(reinterpret_cast<const float4*>(p + (h0 + u) * hs));
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        if (h0 + u < n_heads) {
+          s.x += v[u].x;
+          s.y += v[u].y;
+          s.z += v[u].z;
+          s.w += v[u].w;
+        }
+    }
+    const float sc = 1.0f / (float)(n * n_heads);
+    s.x *= sc;
+    s.y *= sc;
+    s.z *= sc;
+    s.w *= sc;
+  }
+  *reinterpret_cast<float4*>(mass + (size_t)b * plan.row_stride + j) = s;
+}
+
 // Order-preserving map of a float to an unsigned key (larger float, larger key).
 __device__ __forceinline__ uint32_t fkey(float f) {
   const uint32_t u = __float_as_uint(f);
@@ -39,6 +76,7 @@ __device__ __forceinline__ uint32_t fkey(float f) {
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_MAXK = 1024;
 constexpr int SEL_MAXL = 65536;
+constexpr int SEL_SMEM_KEYS = 5120;   // rows up to this length keep their keys on chip
 
 // One CTA per sequence. Exact radix select of the k-th largest key (4 passes
 // of 8 bits), then the strictly larger keys plus the lowest-slot ties, then a
@@ -63,6 +101,11 @@ __global__ void __launch_bounds__(SEL_THREADS)
   __shared__ uint32_t sk[SEL_MAXK];
   __shared__ int ss[SEL_MAXK];
   __shared__ int warp_sums[SEL_THREADS / 32];
+  __shared__ uint32_t skey[SEL_SMEM_KEYS];
+  const bool staged = L <= SEL_SMEM_KEYS;
+  if (staged)
+    for (int j = tid; j < L; j += SEL_THREADS) skey[j] = fkey(__ldg(m + j));
+  auto key_of = [&](int j) -> uint32_t { return staged ? skey[j] : fkey(__ldg(m + j)); };
 
   for (int i = tid; i < (L + 31) / 32; i += SEL_THREADS) excl[i] = 0u;
   __syncthreads();
@@ -75,11 +118,13 @@ __global__ void __launch_bounds__(SEL_THREADS)
   }
   if (tid == 0) s_total = 0;
   __syncthreads();
-  // candidate count
+  // candidate count (one shared atomic per warp)
   {
     int c = 0;
     for (int j = tid; j < L; j += SEL_THREADS) c += ((excl[j >> 5] >> (j & 31)) & 1u) ? 0 : 1;
-    atomicAdd(&s_total, c);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if ((tid & 31) == 0 && c) atomicAdd(&s_total, c);
   }
   __syncthreads();
   const int total = s_total;
@@ -91,20 +136,54 @@ __global__ void __launch_bounds__(SEL_THREADS)
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += SEL_THREADS) hist[i] = 0;
       __syncthreads();
-      for (int j = tid; j < L; j += SEL_THREADS) {
-        if ((excl[j >> 5] >> (j & 31)) & 1u) continue;
-        const uint32_t key = fkey(m[j]);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      for (int base = 0; base < L; base += SEL_THREADS) {
+        const int j = base + tid;
+        bool in = false;
+        uint32_t dig = 0u;
+        if (j < L && !((excl[j >> 5] >> (j & 31)) & 1u)) {
+          const uint32_t key = key_of(j);
+          in = (key & pmask) == prefix;
+          dig = (key >> shift) & 255u;
+        }
+        // one shared atomic per distinct digit in the warp (keys cluster in
+        // few digits, e.g. a shared exponent byte)
+        const uint32_t act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t same = __match_any_sync(act, dig);
+          if ((tid & 31) == __ffs(same) - 1) atomicAdd(&hist[dig], __popc(same));
+        }
       }
       __syncthreads();
-      if (tid == 0) {
-        int cum = 0, d = 255;
-        for (; d > 0; --d) {
-          if (cum + hist[d] >= remaining) break;
-          cum += hist[d];
+      if (tid < 32) {
+        // the digit (scanning down from 255) at which the count of keys
+        // above reaches `remaining`: lane l holds digits 255-8l .. 248-8l
+        int c[8], sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          c[q] = hist[255 - 8 * tid - q];
+          sum += c[q];
         }
-        s_prefix = prefix | ((uint32_t)d << shift);
-        s_remaining = remaining - cum;
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += t;
+        }
+        const int ex = incl - sum;
+        const uint32_t ball = __ballot_sync(0xffffffffu, ex < remaining && incl >= remaining);
+        if (ball != 0u && tid == __ffs(ball) - 1) {
+          int cum = ex, d = 248 - 8 * tid;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (cum + c[q] >= remaining) {
+              d = 255 - 8 * tid - q;
+              break;
+            }
+            cum += c[q];
+          }
+          s_prefix = prefix | ((uint32_t)d << shift);
+          s_remaining = remaining - cum;
+        }
       }
       __syncthreads();
       prefix = s_prefix;
@@ -120,7 +199,7 @@ __global__ void __launch_bounds__(SEL_THREADS)
   __syncthreads();
   for (int j = tid; j < L; j += SEL_THREADS) {
     if ((excl[j >> 5] >> (j & 31)) & 1u) continue;
-    const uint32_t key = fkey(m[j]);
+    const uint32_t key = key_of(j);
     if (all || key > prefix) {
       const int p = atomicAdd(&s_cnt, 1);
       sk[p] = key;
@@ -135,7 +214,7 @@ __global__ void __launch_bounds__(SEL_THREADS)
     for (int base = 0; base < L; base += SEL_THREADS) {
       const int j = base + tid;
       int f = 0;
-      if (j < L && !((excl[j >> 5] >> (j & 31)) & 1u) && fkey(m[j]) == prefix) f = 1;
+      if (j < L && !((excl[j >> 5] >> (j & 31)) & 1u) && key_of(j) == prefix) f = 1;
       // inclusive scan of f across the block
       int v = f;
       for (int o = 1; o < 32; o <<= 1) {
@@ -145,12 +224,13 @@ __global__ void __launch_bounds__(SEL_THREADS)
       if ((tid & 31) == 31) warp_sums[tid >> 5] = v;
       __syncthreads();
       if (tid < 32) {
-        int w = warp_sums[tid];
+        constexpr int NW = SEL_THREADS / 32;
+        int w = tid < NW ? warp_sums[tid] : 0;
         for (int o = 1; o < 32; o <<= 1) {
           const int t = __shfl_up_sync(0xffffffffu, w, o);
           if (tid >= o) w += t;
         }
-        warp_sums[tid] = w;
+        if (tid < NW) warp_sums[tid] = w;
       }
       __syncthreads();
       const int excl_before = (tid >= 32 ? warp_sums[(tid >> 5) - 1] : 0) + v - f;
@@ -203,8 +283,14 @@ __global__ void __launch_bounds__(SEL_THREADS)
 
 cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
                                cudaStream_t stream) {
-  dim3 grid((plan.row_stride + 255) / 256, plan.batch);
-  mass_reduce_kernel<<<grid, 256, 0, stream>>>(plan, part, mass, n_heads);
+  if (plan.row_stride % 4 == 0 && (reinterpret_cast<uintptr_t>(mass) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(part) & 15) == 0) {
+    dim3 grid((plan.row_stride / 4 + 63) / 64, plan.batch);
+    mass_reduce4_kernel<<<grid, 64, 0, stream>>>(plan, part, mass, n_heads);
+  } else {
+    dim3 grid((plan.row_stride + 255) / 256, plan.batch);
+    mass_reduce_kernel<<<grid, 256, 0, stream>>>(plan, part, mass, n_heads);
+  }
   return cudaGetLastError();
 }
 

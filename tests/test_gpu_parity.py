@@ -148,7 +148,7 @@ def test_two_views_isolated_bitwise_on_gpu():
 
 def test_select_tracked_matches_oracle_exactly():
     rng = np.random.default_rng(7)
-    for trial in range(6):
+    for trial in range(12):
         B = int(rng.integers(1, 9))
         stride = int(rng.choice([64, 300, 1024, 4096, 9000]))
         k = int(rng.choice([1, 8, 32, 64, 200, 1024]))
@@ -157,6 +157,11 @@ def test_select_tracked_matches_oracle_exactly():
         mass = (rng.integers(0, 50, (B, stride)) / 997.0).astype(np.float32)
         if trial % 2:
             mass = rng.random((B, stride)).astype(np.float32)
+        if trial == 10:      # every key equal: the k lowest slots, in order
+            mass = np.full((B, stride), 1e-3, np.float32)
+        if trial == 11:      # mostly zeros, a few distinct values on top
+            mass = np.zeros((B, stride), np.float32)
+            mass[:, ::97] = rng.random((B, len(range(0, stride, 97)))).astype(np.float32)
         ex = [rng.choice(max(int(L), 1), size=min(int(L), 5), replace=False) if L else np.zeros(0, int) for L in lens]
         ex_cu = np.zeros(B + 1, np.int32)
         ex_cu[1:] = np.cumsum([len(e) for e in ex])
@@ -166,6 +171,18 @@ def test_select_tracked_matches_oracle_exactly():
                                       torch.from_numpy(ex_cu).to(dev), torch.from_numpy(ex_s).to(dev)).cpu().numpy()
         ref = O.select_tracked(mass, lens, k, ex_cu, ex_s)
         assert np.array_equal(got, ref), trial
+
+
+def test_fp32_page_size_not_a_multiple_of_four():
+    """A page size of 6 gives mass rows whose length is not a multiple of 4:
+    the mass reduction then takes its one-slot-per-thread form."""
+    sh = W.LayerShape("f32", 128, 2, 64, 6, 10000.0)
+    spec = W.WorkloadSpec("f32_page6", sh, batch=3, kind="divergent", ctx_min=20, ctx_max=40,
+                          window=8, tracked=8, track_k=5, spare_pages=2)
+    meta, x, w, kp, vp = build_inputs(spec, 0)
+    assert (meta.max_blocks * sh.page_size) % 4 != 0
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    check_dense(spec, meta, x, w, kp, vp, g)
 
 
 def test_device_bounds_errors_are_reported_not_trapped():
