@@ -28,6 +28,9 @@ Readings where the pages are silent (each is listed in the design notes):
   * The per-key attention mass is the mean over heads and over the
     sequence's query rows of the softmax probabilities, so it sums to 1.
   * Top-k ties go to the lower slot.
+  * Flash-Verify: the views agree when the mask view's most likely token
+    (lowest id among equal logits) is the drafted token; the confidence is
+    that token's softmax probability; the threshold is a parameter.
 
 Every function here has a pin in tests/test_oracle_pins.py (brute force,
 closed forms, library special cases or invariants); none is "parity
@@ -261,4 +264,47 @@ def select_tracked(mass: np.ndarray, seq_lens, k: int, exclude_cu=None, exclude_
         order = np.lexsort((cand, -vals))      # by -mass, then by slot
         take = cand[order[:k]]
         out[b, :len(take)] = take
+    return out
+
+
+# --------------------------------------------------------------------------
+# Flash-Verify acceptance  [FD ¶3]
+# --------------------------------------------------------------------------
+
+def verify_rows(logits_bits: np.ndarray, dtype: str):
+    """Mask-view prediction and confidence of every row of logits [R, V]:
+    the prediction is the token with the largest logit (the lowest token id
+    among equal largest logits) and the confidence is that token's softmax
+    probability, 1 / sum_v exp(logit_v - max). Computed in float64 from the
+    exactly decoded logits. Returns (pred int32 [R], conf float64 [R])."""
+    lg = decode(logits_bits, dtype)
+    R = lg.shape[0]
+    pred = np.zeros(R, dtype=np.int32)
+    conf = np.zeros(R, dtype=np.float64)
+    for r in range(R):
+        row = lg[r]
+        mx = row.max()
+        pred[r] = int(np.flatnonzero(row == mx)[0])
+        conf[r] = 1.0 / np.sum(np.exp(row - mx))
+    return pred, conf
+
+
+def verify_accept(pred, conf, draft_tokens, cu_rows, tau: float):
+    """Accepted prefix length of every sequence [FD ¶3]: the rows of sequence
+    b are its block positions in causal order; position i is accepted when
+    the mask view's prediction equals the drafted token and its confidence
+    exceeds tau, and acceptance stops at the first position that is not.
+    The confidences are compared as given (a kernel's fp32 values are
+    compared in fp32), so the decision is taken in the kernel's precision.
+    Returns int32 [B]."""
+    B = len(cu_rows) - 1
+    out = np.zeros(B, dtype=np.int32)
+    for b in range(B):
+        n = 0
+        for i in range(int(cu_rows[b]), int(cu_rows[b + 1])):
+            if int(pred[i]) == int(draft_tokens[i]) and conf[i] > tau:
+                n += 1
+            else:
+                break
+        out[b] = n
     return out
