@@ -218,6 +218,28 @@ FDLLM_API fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, v
                                       const int32_t* block_table, const int8_t* view_mask,
                                       float* out, float* attn_mass, void* stream);
 
+/* Flash-Verify acceptance ([FD] paragraph 3: a block position is accepted
+ * only when the draft view and the mask view agree and the mask view's
+ * confidence exceeds a threshold, in causal order, stopping at the first
+ * position that fails).
+ *   mask_logits: DEVICE [rows][vocab] of `dtype` (FDLLM_BF16 or FDLLM_F32):
+ *     the mask view's logits at the block positions; the rows of sequence b
+ *     are cu_rows[b] .. cu_rows[b+1]-1, in position order. Logits must be
+ *     finite or -inf, with at least one finite value per row.
+ *   cu_rows: DEVICE int32 [batch+1], non-decreasing, within [0, rows].
+ *   draft_tokens: DEVICE int32 [rows], the drafted token at each position.
+ *   tau: confidence threshold; acceptance needs conf > tau (compared in fp32).
+ *   pred: DEVICE int32 [rows] out: the most likely token (lowest id among
+ *     equal largest logits).
+ *   conf: DEVICE fp32 [rows] out: that token's softmax probability.
+ *   n_accepted: DEVICE int32 [batch] out: the length of the accepted prefix
+ *     (positions i with pred == draft and conf > tau, from the first on).
+ * Reads the logits once; two launches, asynchronous on `stream`. */
+FDLLM_API fdllm_status fdllm_verify_accept(const void* mask_logits, int32_t dtype, int32_t rows,
+                                 int32_t vocab, const int32_t* cu_rows, int32_t batch,
+                                 const int32_t* draft_tokens, float tau, int32_t* pred,
+                                 float* conf, int32_t* n_accepted, void* stream);
+
 /* Synchronises `stream`, reads and clears the handle's device error word.
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
  * FDLLM_ERR_CUDA. */
@@ -230,8 +252,8 @@ FDLLM_API const char* fdllm_status_string(fdllm_status status);
 FDLLM_API const char* fdllm_last_error(void);
 
 /* Number of kernel launches the last successful fdllm_layer_step,
- * fdllm_layer_step_noalloc or fdllm_select_tracked call on this thread
- * enqueued. */
+ * fdllm_layer_step_noalloc, fdllm_select_tracked or fdllm_verify_accept call
+ * on this thread enqueued. */
 FDLLM_API int32_t fdllm_last_launch_count(void);
 
 #ifdef __cplusplus

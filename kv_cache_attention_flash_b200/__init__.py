@@ -25,7 +25,7 @@ from ._lib import (FDLLM_BF16, FDLLM_F32, FDLLM_OK, CacheConfig, FdllmError, Ste
 
 __all__ = [
     "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_layer_step_noalloc",
-    "fdllm_select_tracked",
+    "fdllm_select_tracked", "fdllm_verify_accept",
     "fdllm_check", "fdllm_last_launch_count", "FlashCache", "FdllmError", "load",
 ]
 
@@ -159,6 +159,34 @@ def fdllm_select_tracked(attn_mass: torch.Tensor, seq_lens: torch.Tensor, k: int
         _dev_ptr(exclude_slots, torch.int32, "exclude_slots"), _dev_ptr(tracked, torch.int32, "tracked"),
         _stream_ptr(stream)))
     return tracked
+
+
+def fdllm_verify_accept(mask_logits: torch.Tensor, cu_rows: torch.Tensor,
+                        draft_tokens: torch.Tensor, tau: float, pred: Optional[torch.Tensor] = None,
+                        conf: Optional[torch.Tensor] = None,
+                        n_accepted: Optional[torch.Tensor] = None, stream=None):
+    """Flash-Verify acceptance (see include/fdllm.h): returns (pred, conf,
+    n_accepted) for mask-view logits [rows, vocab] (bf16 or fp32)."""
+    lib = load()
+    if mask_logits.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("mask_logits must be bf16 or fp32")
+    rows, vocab = mask_logits.shape
+    batch = int(cu_rows.numel()) - 1
+    dev = mask_logits.device
+    if pred is None:
+        pred = torch.empty(rows, dtype=torch.int32, device=dev)
+    if conf is None:
+        conf = torch.empty(rows, dtype=torch.float32, device=dev)
+    if n_accepted is None:
+        n_accepted = torch.empty(batch, dtype=torch.int32, device=dev)
+    check_status(lib.fdllm_verify_accept(
+        _dev_ptr(mask_logits, None, "mask_logits"),
+        FDLLM_BF16 if mask_logits.dtype == torch.bfloat16 else FDLLM_F32, int(rows), int(vocab),
+        _dev_ptr(cu_rows, torch.int32, "cu_rows"), batch,
+        _dev_ptr(draft_tokens, torch.int32, "draft_tokens"), float(tau),
+        _dev_ptr(pred, torch.int32, "pred"), _dev_ptr(conf, torch.float32, "conf"),
+        _dev_ptr(n_accepted, torch.int32, "n_accepted"), _stream_ptr(stream)))
+    return pred, conf, n_accepted
 
 
 def fdllm_check(handle: int, stream=None) -> None:

@@ -481,6 +481,26 @@ fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_t* seq_len
   return FDLLM_OK;
 }
 
+fdllm_status fdllm_verify_accept(const void* mask_logits, int32_t dtype, int32_t rows,
+                                 int32_t vocab, const int32_t* cu_rows, int32_t batch,
+                                 const int32_t* draft_tokens, float tau, int32_t* pred,
+                                 float* conf, int32_t* n_accepted, void* stream) {
+  if (dtype != FDLLM_BF16 && dtype != FDLLM_F32)
+    return fail(FDLLM_ERR_INVALID_ARG, "verify_accept: unknown dtype %d", dtype);
+  if (rows < 0 || batch <= 0 || vocab <= 0)
+    return fail(FDLLM_ERR_INVALID_ARG, "verify_accept: rows >= 0, batch > 0, vocab > 0 required");
+  if (!cu_rows || !n_accepted)
+    return fail(FDLLM_ERR_INVALID_ARG, "verify_accept: null cu_rows or n_accepted");
+  if (rows > 0 && (!mask_logits || !draft_tokens || !pred || !conf))
+    return fail(FDLLM_ERR_INVALID_ARG, "verify_accept: null logits, draft tokens, pred or conf");
+  cudaError_t e = launch_verify_accept(mask_logits, dtype == FDLLM_BF16, rows, vocab, cu_rows,
+                                       batch, draft_tokens, tau, pred, conf, n_accepted,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "verify_accept: launch");
+  g_last_launches = rows > 0 ? 2 : 1;
+  return FDLLM_OK;
+}
+
 fdllm_status fdllm_check(fdllm_cache* h, void* stream) {
   if (!h) return fail(FDLLM_ERR_INVALID_ARG, "check: null handle");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

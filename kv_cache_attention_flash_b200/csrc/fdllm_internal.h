@@ -75,6 +75,11 @@ cudaError_t launch_select_tracked(const float* mass, const int32_t* seq_lens, in
                                   const int32_t* exclude_slots, int32_t* tracked,
                                   cudaStream_t stream);
 
+cudaError_t launch_verify_accept(const void* logits, bool bf16, int rows, int vocab,
+                                 const int32_t* cu_rows, int batch, const int32_t* draft,
+                                 float tau, int32_t* pred, float* conf, int32_t* n_accepted,
+                                 cudaStream_t stream);
+
 size_t step_bf16_smem_bytes();
 
 }  // namespace fdllm

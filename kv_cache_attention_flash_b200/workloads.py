@@ -359,3 +359,58 @@ def algorithmic_bytes_flops(spec: WorkloadSpec, meta: StepMeta, with_mass: bool 
             keys += k
     fl += 4 * sh.head_dim * sh.n_heads * keys
     return byt, fl
+
+
+# ------------------------------------------------------------------ Flash-Verify
+@dataclasses.dataclass(frozen=True)
+class VerifySpec:
+    """Mask-view logits of a Flash-Verify block for every sequence."""
+    name: str
+    batch: int
+    rows: int            # block positions per sequence (the mask view's rows)
+    vocab: int
+    dtype: str           # "bf16" or "f32"
+    tau: float           # confidence threshold
+
+
+VERIFY_WORKLOADS: Dict[str, VerifySpec] = {
+    # the two-view workload's mask view: batch 8 x 32 positions, LLaDA
+    # vocabulary (126464 tokens), bf16 logits
+    "verify_b8": VerifySpec("verify_b8", batch=8, rows=32, vocab=126464, dtype="bf16", tau=0.9),
+    "verify_small": VerifySpec("verify_small", batch=5, rows=12, vocab=1000, dtype="bf16", tau=0.6),
+}
+
+
+def make_verify(spec: VerifySpec, seed: int, device="cpu"):
+    """(logits [R, V], cu_rows [B+1] int32, draft [R] int32).
+
+    Logits are N(0, 2^2). Each sequence gets a seeded prefix length a in
+    [0, rows]; the drafted token of a position before a is given a raised
+    logit (+9 to +14, so that it is usually the most likely token with a
+    high softmax probability), the position at a gets a draft token with no
+    raised logit (or a smaller raise), and later positions get random
+    drafts, half of them raised. The step's own rule then decides what is
+    accepted."""
+    rng = np.random.default_rng(seed)
+    B, n, V = spec.batch, spec.rows, spec.vocab
+    R = B * n
+    g = _gen(seed * 1000003 + 57, device)
+    logits = torch.randn(R, V, generator=g, device=device, dtype=torch.float32) * 2.0
+    draft = rng.integers(0, V, R).astype(np.int64)
+    boost = np.zeros(R)
+    for b in range(B):
+        a = int(rng.integers(0, n + 1))
+        for i in range(n):
+            r = b * n + i
+            if i < a:
+                boost[r] = rng.uniform(9.0, 14.0)
+            elif i == a:
+                boost[r] = 0.0 if rng.random() < 0.5 else rng.uniform(1.0, 4.0)
+            else:
+                boost[r] = rng.uniform(9.0, 14.0) if rng.random() < 0.5 else 0.0
+    rows_t = torch.arange(R, device=device)
+    d_t = torch.from_numpy(draft).to(device)
+    logits[rows_t, d_t] += torch.from_numpy(boost).to(device=device, dtype=torch.float32)
+    dt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    cu = (np.arange(B + 1) * n).astype(np.int32)
+    return logits.to(dt), cu, draft.astype(np.int32)
