@@ -2,6 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
+`--workload verify_b8` measures the Flash-Verify acceptance step instead
+(mask-view logits of 8 x 32 block positions over the 126464-token LLaDA
+vocabulary, bf16): positions/s, HBM roofline of the logits read.
+
 A step is one pass of the whole hot path over one batch of synthetic input:
 the fused layer step (projection, RoPE, cache write, scheduled attention,
 attention mass) for every layer of the workload, then the top-k tracking
@@ -473,12 +477,185 @@ def run_native(args):
     return 0
 
 
+# ------------------------------------------------------------------ Flash-Verify
+VERIFY_METRIC = "Flash-Verify acceptance block-positions/s; achieved HBM GB/s and % of roofline (1×B200)"
+VERIFY_UNIT = "positions/s"
+
+
+def verify_bytes(spec):
+    """Algorithmic bytes of one acceptance step: the logits once, the drafted
+    tokens, predictions and confidences (4 bytes each per row), cu_rows and
+    the accepted lengths."""
+    s = 2 if spec.dtype == "bf16" else 4
+    R = spec.batch * spec.rows
+    return R * spec.vocab * s + R * 12 + (spec.batch + 1) * 4 + spec.batch * 4
+
+
+def verify_oracle_sample(spec, logits_cpu, cu, draft, budget_s):
+    from oracle import oracle as O
+    bits = W.bits_np(logits_cpu)
+    t0 = time.perf_counter()
+    rows = 0
+    nseq = 0
+    while nseq < spec.batch and time.perf_counter() - t0 < budget_s:
+        r0, r1 = int(cu[nseq]), int(cu[nseq + 1])
+        pred, conf = O.verify_rows(bits[r0:r1], spec.dtype)
+        O.verify_accept(pred, conf, draft[r0:r1], np.array([0, r1 - r0]), spec.tau)
+        rows += r1 - r0
+        nseq += 1
+    dt = time.perf_counter() - t0
+    desc = (f"oracle (numpy float64) on {nseq} of {spec.batch} sequences ({rows} positions x "
+            f"{spec.vocab} logits), one sequence per call, {dt:.1f} s")
+    return rows / dt, desc
+
+
+def verify_config(spec, args, world):
+    return {"workload": spec.name, "batch": spec.batch, "positions_per_sequence": spec.rows,
+            "vocab": spec.vocab, "logits": spec.dtype, "tau": spec.tau,
+            "l2": "flushed between timed steps (256 MB write)", "parallelism": f"replicas x{world}",
+            "seed": args.seed}
+
+
+def run_verify(args):
+    rank, world, local = dist_env()
+    spec = W.VERIFY_WORKLOADS[args.workload]
+    R = spec.batch * spec.rows
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        logits, cu, draft = W.make_verify(spec, args.seed)
+        budget = max(2.0, 20.0 / max(1, args.steps + args.warmup))
+        vals, desc = [], ""
+        for i in range(args.warmup + args.steps):
+            v, desc = verify_oracle_sample(spec, logits, cu, draft, budget)
+            if i >= args.warmup:
+                vals.append(v)
+        value = float(np.mean(vals))
+        line = {"impl": "reference", "metric": VERIFY_METRIC, "value": value, "unit": VERIFY_UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * R / value, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": verify_config(spec, args, args.gpus),
+                "cpu_baseline": {"value": value, "unit": VERIFY_UNIT, "cores": os.cpu_count() or 1,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": value, "unit": VERIFY_UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+    import kv_cache_attention_flash_b200 as fd
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    logits, cu, draft = W.make_verify(spec, args.seed + rank, device=dev)
+    cu_d = torch.from_numpy(cu).to(dev)
+    draft_d = torch.from_numpy(draft).to(dev)
+    pred = torch.empty(R, dtype=torch.int32, device=dev)
+    conf = torch.empty(R, dtype=torch.float32, device=dev)
+    nacc = torch.empty(spec.batch, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fd.fdllm_verify_accept(logits, cu_d, draft_d, spec.tau, pred, conf, nacc)
+        return fd.fdllm_last_launch_count()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev_s[i].record()
+        launches += step()
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    if sampler:
+        sampler.mark(t_wall0, t_wall1)
+        time.sleep(0.25)
+        sampler.stop()
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    total_ms, _, value = aggregate(float(sum(step_ms)), R * args.steps, dev)
+    byt = verify_bytes(spec)
+    kern_s = float(np.mean(step_ms)) / 1000.0
+    achieved = byt / kern_s / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} (burst)",
+            "kernel": "fdllm_verify_accept (row reduction + acceptance scan)",
+            "kernel_us": kern_s * 1e6, "algorithmic_bytes": byt}
+    # end to end: logits from pinned host memory in, predictions,
+    # confidences and accepted lengths out, every step
+    hlog = logits.cpu().pin_memory()
+    hpred = torch.empty(R, dtype=torch.int32).pin_memory()
+    hconf = torch.empty(R, dtype=torch.float32).pin_memory()
+    hnacc = torch.empty(spec.batch, dtype=torch.int32).pin_memory()
+    dlog = torch.empty_like(logits)
+    h2d = hlog.numel() * hlog.element_size()
+    d2h = R * 8 + spec.batch * 4
+    n_e2e = max(10, min(args.steps, 200))
+
+    def one():
+        dlog.copy_(hlog, non_blocking=True)
+        fd.fdllm_verify_accept(dlog, cu_d, draft_d, spec.tau, pred, conf, nacc)
+        hpred.copy_(pred, non_blocking=True)
+        hconf.copy_(conf, non_blocking=True)
+        hnacc.copy_(nacc, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, dev)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc = verify_oracle_sample(spec, logits.cpu(), cu, draft, 12.0)
+        cpu = {"value": v, "unit": VERIFY_UNIT, "cores": os.cpu_count() or 1, "kind": "oracle",
+               "sample": desc}
+    line = {
+        "metric": VERIFY_METRIC, "value": value, "unit": VERIFY_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": spec.dtype,
+        "data": "synthetic", "config": verify_config(spec, args, world), "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": R * world / (e2e_ms / 1000.0), "unit": VERIFY_UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches, "clocks": sampler.summary() if sampler else None,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="b32_divergent", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="b32_divergent",
+                    choices=sorted(W.WORKLOADS) + sorted(W.VERIFY_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
@@ -487,6 +664,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload in W.VERIFY_WORKLOADS:
+        return run_verify(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_native(args)

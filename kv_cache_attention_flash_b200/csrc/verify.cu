@@ -23,7 +23,7 @@
 namespace fdllm {
 namespace {
 
-constexpr int VT = 256;                 // threads per row
+constexpr int VT = 512;                 // threads per row
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Acc {
@@ -55,6 +55,54 @@ __device__ __forceinline__ void merge(Acc& a, Acc b) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// N consecutive logits (indices e0 .. e0+N-1) at once: their maximum first
+// (at most one rescale of the running sum), then N independent exponentials
+// added as a tree, so a thread keeps N exponentials in flight.
+template <int N>
+__device__ __forceinline__ void push_n(Acc& a, const float* v, int e0) {
+  float lm = v[0];
+  int li = 0;
+#pragma unroll
+  for (int i = 1; i < N; ++i)
+    if (v[i] > lm) {
+      lm = v[i];
+      li = i;
+    }
+  if (lm > a.m) {
+    a.s *= ptx::ex2((a.m - lm) * kLog2e);   // a.m = -inf: 0
+    a.m = lm;
+    a.idx = e0 + li;
+  }
+  if (a.m == -INFINITY) return;             // nothing finite seen yet
+  const float mc = a.m * kLog2e;
+  float t[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) t[i] = ptx::ex2(fmaf(v[i], kLog2e, -mc));
+#pragma unroll
+  for (int w = N / 2; w > 0; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] += t[i + w];
+  a.s += t[0];
+}
+
+__device__ __forceinline__ void push_vec(Acc& a, const uint4& w, int e0, bool bf16) {
+  const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+  if (bf16) {
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = bf16_lo(q[k]);
+      v[2 * k + 1] = bf16_hi(q[k]);
+    }
+    push_n<8>(a, v, e0);
+  } else {
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = __uint_as_float(q[k]);
+    push_n<4>(a, v, e0);
+  }
+}
+
 template <bool kBf16>
 __global__ void __launch_bounds__(VT) verify_rows_kernel(const void* logits, int vocab,
                                                          int32_t* pred, float* conf) {
@@ -76,36 +124,9 @@ __global__ void __launch_bounds__(VT) verify_rows_kernel(const void* logits, int
 #pragma unroll
       for (int u = 0; u < U; ++u) w[u] = __ldg(v4 + i + u * VT);
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int e0 = (i + u * VT) * EPV;
-        const uint32_t q[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-        if (kBf16) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            push(a, bf16_lo(q[k]), e0 + 2 * k);
-            push(a, bf16_hi(q[k]), e0 + 2 * k + 1);
-          }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) push(a, __uint_as_float(q[k]), e0 + k);
-        }
-      }
+      for (int u = 0; u < U; ++u) push_vec(a, w[u], (i + u * VT) * EPV, kBf16);
     }
-    for (; i < nvec; i += VT) {
-      const uint4 w = __ldg(v4 + i);
-      const int e0 = i * EPV;
-      const uint32_t q[4] = {w.x, w.y, w.z, w.w};
-      if (kBf16) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          push(a, bf16_lo(q[k]), e0 + 2 * k);
-          push(a, bf16_hi(q[k]), e0 + 2 * k + 1);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) push(a, __uint_as_float(q[k]), e0 + k);
-      }
-    }
+    for (; i < nvec; i += VT) push_vec(a, __ldg(v4 + i), i * EPV, kBf16);
     done = nvec * EPV;
   }
   // the rest one element at a time (all of an unaligned row)
