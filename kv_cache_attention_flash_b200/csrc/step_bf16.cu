@@ -197,10 +197,13 @@ __device__ __forceinline__ void epi_q(uint32_t taddr, int qrow, bool valid, int 
 }
 
 // k (rotated) or v (plain) rows -> bf16 staging rows for the cache copy.
+// Pass c covers dimensions [32c, 32c + 32) and [64 + 32c, 64 + 32c + 32)
+// (the rotate-half pairs); passes [c0, c1) are done.
 __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool rotate, int pos,
-                                       const float* cos_t, const float* sin_t, uint8_t* dst) {
+                                       const float* cos_t, const float* sin_t, uint8_t* dst,
+                                       int c0 = 0, int c1 = 2) {
 #pragma unroll 1
-  for (int c = 0; c < 2; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float lo[32], hi[32];
     ptx::tmem_ld32(taddr + 32 * c, lo);
     ptx::tmem_ld32(taddr + 64 + 32 * c, hi);
@@ -520,13 +523,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const bool valid = acc_ok && ctrl->row_page[i] >= 0;
     const int pos = ctrl->row_pos[i];
     const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+    // warps 0-3: q and the first v pass; warps 4-7: k and the second v
+    // pass (v needs no rotation, so the halves balance)
     if (warp >= 8) {
       // producer and MMA warps take no part in the epilogue
     } else if (warp < 4) {
       epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
+      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, 0, 1);
     } else {
       epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF);
-      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF);
+      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, 1, 2);
     }
   }
   ptx::tc_fence_before();
