@@ -74,6 +74,10 @@ constexpr int NSLOT = 3;
 constexpr int PT_OFF = SLOT_OFF + NSLOT * SLOT_BYTES;   // P^T hi, then lo
 constexpr int PT_BYTES = 32768;       //   core matrices: [rows/8][128 keys][16 B]
 static_assert(PT_OFF + 2 * PT_BYTES <= PIPE_BYTES, "attention buffers overflow");
+// A sequence of at most 64 rows keeps P^T lo at PT_OFF + 16 KB; the last
+// 32 KB then hold its q rows repeated across the four TMEM lane quadrants
+// for pass 1.
+constexpr int QREP_OFF = PT_OFF + 32768;
 
 // TMEM columns during attention.
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
@@ -88,6 +92,7 @@ struct Ctrl {
   uint64_t s_empty[2];
   uint64_t p_full;
   uint64_t pv_done;
+  uint64_t q_ready;       // repeated q rows written (sequences of at most 64 rows)
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
@@ -107,7 +112,7 @@ struct Ctrl {
   short pg_log[MAX_PAGES];  // per sequence: logical pages attended, in order
   int pg_phys[MAX_PAGES];   //   and their physical pages (-1: bad table entry)
   alignas(16) float lse2[BM];   // log2-sum-exp2 of the scaled scores of each row (float4 loads)
-  float pm[BM], pl[BM];          // pass-1 partial (max, sum) of the second key half
+  float pm2[2][BM], pl2[2][BM];  // pass-1 partial (max, sum) per TMEM lane and warp half
 };
 static_assert(offsetof(Ctrl, lse2) % 16 == 0, "lse2 is read as float4");
 static_assert(sizeof(Ctrl) % 16 == 0 || true, "");
@@ -263,6 +268,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ptx::mbar_init(&ctrl->mma_done, 1);
     ptx::mbar_init(&ctrl->p_full, 8);
     ptx::mbar_init(&ctrl->pv_done, 1);
+    ptx::mbar_init(&ctrl->q_ready, 8);
     ptx::mbar_init(&ctrl->o_done, 1);
     ctrl->abort = 0;
     ptx::fence_mbar_init();
@@ -570,9 +576,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t q_base = ptx::smem_u32(smem + Q_OFF);
   const uint32_t slot_base = ptx::smem_u32(smem + SLOT_OFF);
   const uint32_t pt_base = ptx::smem_u32(smem + PT_OFF);
+  const uint32_t qrep_base = ptx::smem_u32(smem + QREP_OFF);
   // Schedule counters, identical in every thread: chunk loads (K or V)
-  // issued so far, S^T products, P.V products, finished sequences.
-  uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0;
+  // issued so far, S^T products, P.V products, finished sequences and
+  // sequences whose q rows were repeated.
+  uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0, qcount = 0;
 
   const int nseq_g = ctrl->nseq;
   for (int si = 0; si < nseq_g; ++si) {
@@ -583,7 +591,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int L = ctrl->sq_L[si];
     const int N16 = (n + 15) & ~15;
     const int qoff = ctrl->sq_qoff[si];
-    const int nblk = (N16 + 31) >> 5;
     const int npages = ctrl->sq_npages[si];
     const int nx = ctrl->sq_nx[si];
     const bool any_page = ctrl->sq_any[si] != 0;
@@ -592,6 +599,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int* xsl = ctrl->xs_slot + ctrl->sq_x0[si];
     const int* xsr = ctrl->xs_row + ctrl->sq_x0[si];
     const int nch = (npages + 1) >> 1;
+    // Pass 1 keeps the rows on TMEM lanes. A sequence of at most 64 rows
+    // is repeated R times (copy rho on lanes [rho*RS, rho*RS + N16)), so
+    // that every lane quadrant (every SM sub-partition) holds rows; copy
+    // rho takes the chunk's keys [rho*KR, rho*KR + KR), split between the
+    // two warps of its quadrant. A wider sequence uses the group's q rows.
+    const bool wide = N16 > 64;
+    const int R = N16 <= 32 ? 4 : (N16 <= 64 ? 2 : 1);
+    const int RS = 128 / R;
+    const int KR = 128 / R;
+    const uint32_t ptl_off = wide ? 32768u : 16384u;   // P^T lo after hi
     float* part = a.mass_part ? a.mass_part + ((size_t)h * plan.batch + b) * plan.row_stride
                               : nullptr;
     // Chunk loads of this sequence, in ring order: pass 1 K_0 .. K_{nch-1}
@@ -668,13 +685,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const uint64_t qd = ptx::smem_desc_sw128(q_base + off + qoff * 128, 16, 1024);
               ptx::umma_f16_ss(tmem + (sb ? TM_S1 : TM_S0), kd, qd, idesc_s, kk > 0 ? 1u : 0u);
             } else {
-              const uint64_t qd = ptx::smem_desc_sw128(q_base + off, 16, 1024);
+              const uint64_t qd = ptx::smem_desc_sw128((wide ? q_base : qrep_base) + off, 16, 1024);
               ptx::umma_f16_ss(tmem + (sb ? TM_S1 : TM_S0), qd, kd, idesc_std, kk > 0 ? 1u : 0u);
             }
           }
           ptx::umma_commit(&ctrl->s_full[sb]);
           ptx::umma_commit(&ctrl->aempty[s]);
         };
+        if (!wide) wait_bar(ctrl, &ctrl->q_ready, qcount & 1, a.err, 16);
         for (int c = 0; c < nch; ++c) issue_s(c, r0 + c, false);
         for (int c = 0; c < npre; ++c) issue_s(nch + c, item_k2(c), true);
         bool any = false;
@@ -698,7 +716,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               // B = P^T: N-major core matrices without swizzle: 8-key
               // groups 128 B apart (LBO), 8-row blocks 2048 B apart (SBO).
               const uint64_t bh = ptx::smem_desc_noswz(pt_base + ks * 256, 128, 2048);
-              const uint64_t bl = ptx::smem_desc_noswz(pt_base + PT_BYTES + ks * 256, 128, 2048);
+              const uint64_t bl = ptx::smem_desc_noswz(pt_base + ptl_off + ks * 256, 128, 2048);
               ptx::umma_f16_ss(tmem + TM_O, ad, bh, idesc_pv, any ? 1u : 0u);
               ptx::umma_f16_ss(tmem + TM_O, ad, bl, idesc_pv, 1u);
               any = true;
@@ -762,16 +780,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         return m;
       };
 
-      // ----- pass 1: log-sum-exp of every row. S = Q K^T has the group's q
-      // rows on TMEM lanes, so thread t owns q row t; the warp pair of a
-      // quadrant splits the 128 keys of a chunk (half h takes page h), and
-      // the two partial (max, sum) pairs are merged once at the end.
+      // ----- repeated q rows for pass 1 (sequences of at most 64 rows):
+      // lane t holds row t % RS. A 128-byte row's swizzle phase depends on
+      // its index mod 8, which the copy preserves, so rows copy verbatim.
+      if (!wide) {
+        for (int i = tid; i < 128 * 16; i += NSMX) {
+          const int lt = i >> 4;
+          const int hd = (i >> 3) & 1;
+          const int c8 = i & 7;
+          const int r = lt % RS;
+          if (r >= N16) continue;
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + Q_OFF + hd * HALF_BYTES +
+                                                          (qoff + r) * 128 + c8 * 16);
+          *reinterpret_cast<uint4*>(smem + QREP_OFF + hd * HALF_BYTES + lt * 128 + c8 * 16) = v;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ctrl->q_ready);
+      }
+
+      // ----- pass 1: log-sum-exp of every row. S = Q K^T has rows on TMEM
+      // lanes: thread t owns one row copy and half of the copy's keys of
+      // every chunk (KR / 2 of them), keeping a running max and sum; the
+      // partial pairs of all copies and both halves are merged at the end.
       {
-        const int r = t - qoff;                    // sequence row of q row t
+        const int rho = wide ? 0 : t / RS;
+        const int r = wide ? t - qoff : t - rho * RS;   // sequence row of lane t
         const bool active = r >= 0 && r < n;
         const bool warp_active = __any_sync(0xffffffffu, active);
         const int myview = active ? ctrl->row_view[ra + r] : 0;
         const int mypos = active ? ctrl->row_pos[ra + r] : 0;
+        const int KH = KR >> 1;                      // keys per thread per chunk
+        const int jbeg = rho * KR + half * KH;       // first chunk column of this thread
         float m = -INFINITY, l = 0.f;
         for (int c = 0; c < nch; ++c) {
           const uint32_t idx = s0 + c;
@@ -779,31 +819,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 20);
           ptx::tc_fence_after();
           if (warp_active) {
-            // keys of this warp's page of the chunk that this row attends:
-            // context slots, then view slots of its own view at positions
-            // <= its own
-            uint64_t km = 0ull;
-            const int pidx = 2 * c + half;
-            if (pidx < npages && pgp[pidx] >= 0) {
-              const int plog = (int)pgl[pidx];
-              const int nv = min(max(L - plog * PS, 0), PS);
-              km = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-              if (nv < PS && myview != 0) {
-                for (int x = 0; x < nx; ++x) {
-                  const int xs = xsl[x];
-                  const int xr = xsr[x];
-                  if (xs / PS == plog && ctrl->row_view[xr] == myview && ctrl->row_pos[xr] <= mypos)
-                    km |= 1ull << (xs % PS);
+#pragma unroll 1
+            for (int j0 = jbeg; j0 < jbeg + KH; j0 += 32) {
+              const int nk = KH < 32 ? KH : 32;      // keys in this block (16 or 32)
+              // keys j0 .. j0+nk-1 of the chunk lie in one page, pidx; this
+              // row attends its context slots, then view slots of its own
+              // view at positions <= its own
+              const int pidx = 2 * c + (j0 >> 6);
+              uint64_t km = 0ull;
+              if (pidx < npages && pgp[pidx] >= 0) {
+                const int plog = (int)pgl[pidx];
+                const int nv = min(max(L - plog * PS, 0), PS);
+                km = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+                if (nv < PS && myview != 0) {
+                  for (int x = 0; x < nx; ++x) {
+                    const int xs = xsl[x];
+                    const int xr = xsr[x];
+                    if (xs / PS == plog && ctrl->row_view[xr] == myview &&
+                        ctrl->row_pos[xr] <= mypos)
+                      km |= 1ull << (xs % PS);
+                  }
                 }
               }
-            }
-            if (!active) km = 0ull;
-            const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + 64 * half;
-#pragma unroll 1
-            for (int blk = 0; blk < 2; ++blk) {
+              uint32_t mk = active ? (uint32_t)(km >> (j0 & 63)) : 0u;
+              if (nk < 32) mk &= (1u << nk) - 1u;
               float v[32];
-              ptx::tmem_ld32(sbase + 32 * blk, v);
-              const uint32_t mk = blk ? (uint32_t)(km >> 32) : (uint32_t)km;
+              const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + j0;
+              if (nk == 32) {
+                ptx::tmem_ld32(sbase, v);
+              } else {
+                ptx::tmem_ld16(sbase, v);
+#pragma unroll
+                for (int j = 16; j < 32; ++j) v[j] = -INFINITY;
+              }
               ptx::tmem_ld_wait();
               // four independent max / sum chains
               float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -829,16 +877,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
         }
-        if (half == 1) {
-          ctrl->pm[t] = m;
-          ctrl->pl[t] = l;
-        }
+        ctrl->pm2[half][t] = m;
+        ctrl->pl2[half][t] = l;
         named_bar(1, NSMX);
-        if (half == 0 && active) {
-          const float m1 = ctrl->pm[t], l1 = ctrl->pl[t];
-          const float M = fmaxf(m, m1);
-          const float S = (M == -INFINITY) ? 0.f : l * ptx::ex2(m - M) + l1 * ptx::ex2(m1 - M);
-          ctrl->lse2[r] = S > 0.f ? M + log2f(S) : INFINITY;
+        for (int rr = tid; rr < n; rr += NSMX) {
+          float M = -INFINITY;
+          for (int q = 0; q < R; ++q)
+            for (int hp = 0; hp < 2; ++hp)
+              M = fmaxf(M, ctrl->pm2[hp][wide ? qoff + rr : q * RS + rr]);
+          float S = 0.f;
+          if (M != -INFINITY) {
+            for (int q = 0; q < R; ++q)
+              for (int hp = 0; hp < 2; ++hp) {
+                const int lt = wide ? qoff + rr : q * RS + rr;
+                const float mq = ctrl->pm2[hp][lt];
+                if (mq != -INFINITY) S += ctrl->pl2[hp][lt] * ptx::ex2(mq - M);
+              }
+          }
+          ctrl->lse2[rr] = S > 0.f ? M + log2f(S) : INFINITY;
         }
         named_bar(1, NSMX);
       }
@@ -910,7 +966,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t pidx_g = p0 + c;
         if (pidx_g > 0) wait_bar(ctrl, &ctrl->pv_done, (pidx_g - 1) & 1, a.err, 23);
         uint8_t* pth = smem + PT_OFF;
-        uint8_t* ptl = pth + PT_BYTES;
+        uint8_t* ptl = pth + ptl_off;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int k = 2 * u + half;
@@ -948,6 +1004,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     scount = s0 + 2 * nch;
     pcount = p0 + nch;
     ++ocount;
+    if (!wide) ++qcount;
   }
 
   // ================================================================ teardown
