@@ -21,10 +21,12 @@
 // Phase 3 (attention), per sequence of the group, on the tensor cores. K
 //   and V pages are gathered by TMA through the block table, two 64-slot
 //   pages per 128-key chunk, into a 3-slot ring.
-//   Pass 1 finds every row's log-sum-exp from S = Q K^T (the group's q rows
-//   on TMEM lanes, so each thread keeps its own row's running max and sum;
-//   the two warps of a lane quadrant take one page of the chunk each and
-//   merge once at the end).
+//   Pass 1 finds every row's log-sum-exp from S = Q K^T with the rows on
+//   TMEM lanes, so each thread keeps its own row's running max and sum. A
+//   sequence of at most 64 rows is first repeated across the four lane
+//   quadrants, each copy taking a share of every chunk's keys, so that all
+//   four SM sub-partitions share its exponentials; the two warps of a
+//   quadrant split the copy's keys, and the partial pairs merge at the end.
 //   Pass 2 runs in transposed form so that a sequence of only 16..128 rows
 //   wastes no MMA rows: S^T = K Q^T (keys on lanes, the sequence's rows on
 //   columns) gives the exact probabilities, whose per-key sums over the
