@@ -240,6 +240,34 @@ FDLLM_API fdllm_status fdllm_verify_accept(const void* mask_logits, int32_t dtyp
                                  const int32_t* draft_tokens, float tau, int32_t* pred,
                                  float* conf, int32_t* n_accepted, void* stream);
 
+/* Host-only: the static tile schedule the bf16 layer step uses when its
+ * (row group, head) tiles outnumber the SMs. The step then launches one
+ * persistent CTA per SM (per bin), which runs its bin's tiles one after
+ * another; fdllm_layer_step builds this schedule itself (with the device's
+ * SM count and its own per-group cost model, and caches it while the costs
+ * repeat). This entry point exposes the packing for inspection and tests.
+ *
+ * [FD] paragraph 1 (scheduled attention over divergent lengths and stages
+ * in one launch): the packing balances that launch across SMs; the pages
+ * prescribe no particular packing.
+ *
+ *   group_cost: HOST double [n_groups], the modelled time of one tile of
+ *     group g (every head's tile of a group costs the same); finite, >= 0.
+ *   n_groups, n_heads: tile t = g * n_heads + h for group g, head h.
+ *     At most 256 each, and n_groups * n_heads <= 1024.
+ *   n_bins: number of bins (persistent CTAs), 1 .. 160.
+ *   bin_start: HOST int32 [n_bins + 1] out: bin i runs
+ *     tiles[bin_start[i] .. bin_start[i+1]), costliest first; bin_start[0]
+ *     is 0 and bin_start[n_bins] is n_groups * n_heads.
+ *   tiles: HOST int32 [n_groups * n_heads] out: every tile exactly once.
+ * Packing: first-fit-decreasing into n_bins bins of the smallest capacity
+ * that fits (bisection), then moves and swaps out of the fullest bin while
+ * they lower it. Deterministic. Returns FDLLM_ERR_INVALID_ARG or
+ * FDLLM_ERR_UNSUPPORTED outside these limits; needs no GPU. */
+FDLLM_API fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_t n_groups,
+                                      int32_t n_heads, int32_t n_bins, int32_t* bin_start,
+                                      int32_t* tiles);
+
 /* Synchronises `stream`, reads and clears the handle's device error word.
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
  * FDLLM_ERR_CUDA. */

@@ -25,7 +25,7 @@ from ._lib import (FDLLM_BF16, FDLLM_F32, FDLLM_OK, CacheConfig, FdllmError, Ste
 
 __all__ = [
     "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_layer_step_noalloc",
-    "fdllm_select_tracked", "fdllm_verify_accept",
+    "fdllm_select_tracked", "fdllm_verify_accept", "fdllm_plan_tile_schedule",
     "fdllm_check", "fdllm_last_launch_count", "FlashCache", "FdllmError", "load",
 ]
 
@@ -187,6 +187,21 @@ def fdllm_verify_accept(mask_logits: torch.Tensor, cu_rows: torch.Tensor,
         _dev_ptr(pred, torch.int32, "pred"), _dev_ptr(conf, torch.float32, "conf"),
         _dev_ptr(n_accepted, torch.int32, "n_accepted"), _stream_ptr(stream)))
     return pred, conf, n_accepted
+
+
+def fdllm_plan_tile_schedule(group_cost: Sequence[float], n_heads: int, n_bins: int):
+    """The bf16 step's static tile schedule (see include/fdllm.h): returns
+    (bin_start [n_bins + 1], tiles [n_groups * n_heads]) as int32 arrays;
+    tile t is group t // n_heads, head t % n_heads. Host only."""
+    lib = load()
+    cost = np.ascontiguousarray(np.asarray(group_cost, dtype=np.float64))
+    n_groups = int(cost.size)
+    bin_start = np.zeros(max(int(n_bins), 0) + 1, np.int32)
+    tiles = np.zeros(max(n_groups * int(n_heads), 0), np.int32)
+    check_status(lib.fdllm_plan_tile_schedule(
+        cost.ctypes.data if n_groups else None, n_groups, int(n_heads), int(n_bins),
+        bin_start.ctypes.data, tiles.ctypes.data if tiles.size else None))
+    return bin_start, tiles
 
 
 def fdllm_check(handle: int, stream=None) -> None:

@@ -50,6 +50,7 @@ SIGNATURES = {
     "fdllm_select_tracked": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "fdllm_verify_accept": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _vp, ctypes.c_float, _vp,
                                    _vp, _vp, _vp]),
+    "fdllm_plan_tile_schedule": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "fdllm_check": (_i32, [_vp, _vp]),
     "fdllm_status_string": (ctypes.c_char_p, [_i32]),
     "fdllm_last_error": (ctypes.c_char_p, []),

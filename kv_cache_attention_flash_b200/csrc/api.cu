@@ -8,6 +8,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <queue>
 #include <mutex>
 #include <set>
 #include <string>
@@ -88,6 +89,206 @@ bool encode_wqkv_5d(CUtensorMap* map, const void* base, uint64_t hidden, uint64_
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// First fit of items (in the given order) into P bins of capacity C; the
+// leftmost bin with room is found in a max-tree of remaining capacities.
+bool first_fit(const std::vector<double>& cost, int P, double C, std::vector<int>& bin_of) {
+  int size = 1;
+  while (size < P) size <<= 1;
+  thread_local std::vector<double> tree;
+  tree.assign(2 * size, -1.0);
+  for (int i = 0; i < P; ++i) tree[size + i] = C;
+  for (int i = size - 1; i >= 1; --i) tree[i] = std::max(tree[2 * i], tree[2 * i + 1]);
+  bin_of.assign(cost.size(), -1);
+  for (size_t it = 0; it < cost.size(); ++it) {
+    const double w = cost[it];
+    if (tree[1] < w) return false;
+    int node = 1;
+    while (node < size) node = tree[2 * node] >= w ? 2 * node : 2 * node + 1;
+    bin_of[it] = node - size;
+    tree[node] -= w;
+    for (node >>= 1; node >= 1; node >>= 1) tree[node] = std::max(tree[2 * node], tree[2 * node + 1]);
+  }
+  return true;
+}
+
+// Local improvement of an assignment of items (costs `sorted`) to P bins:
+// while the fullest bin can hand a tile to another bin (or trade it for a
+// cheaper one) and end up below its old load without the other bin reaching
+// it, do the move that lowers the pair's larger load the most. Returns the
+// final largest load.
+double improve_packing(const std::vector<double>& sorted, int P, std::vector<int>& best) {
+  const int n_items = (int)sorted.size();
+  std::vector<double> load(P, 0.0);
+  for (int i = 0; i < n_items; ++i) load[best[i]] += sorted[i];
+  std::vector<std::vector<int>> members(P);
+  for (int i = 0; i < n_items; ++i) members[best[i]].push_back(i);
+  for (int iter = 0; iter < 4 * n_items; ++iter) {
+    const int M = (int)(std::max_element(load.begin(), load.end()) - load.begin());
+    double best_peak = load[M];
+    int bi = -1, bj = -1, bb = -1;
+    for (int ii = 0; ii < (int)members[M].size(); ++ii) {
+      const double wi = sorted[members[M][ii]];
+      for (int b = 0; b < P; ++b) {
+        if (b == M) continue;
+        // move
+        const double pk = std::max(load[M] - wi, load[b] + wi);
+        if (pk < best_peak - 1e-9) {
+          best_peak = pk;
+          bi = ii, bj = -1, bb = b;
+        }
+        // swap with a cheaper tile of bin b
+        for (int jj = 0; jj < (int)members[b].size(); ++jj) {
+          const double wj = sorted[members[b][jj]];
+          if (wj >= wi) continue;
+          const double pk2 = std::max(load[M] - wi + wj, load[b] + wi - wj);
+          if (pk2 < best_peak - 1e-9) {
+            best_peak = pk2;
+            bi = ii, bj = jj, bb = b;
+          }
+        }
+      }
+    }
+    if (bi < 0) break;
+    const int item = members[M][bi];
+    members[M].erase(members[M].begin() + bi);
+    load[M] -= sorted[item];
+    if (bj >= 0) {
+      const int other = members[bb][bj];
+      members[bb].erase(members[bb].begin() + bj);
+      load[bb] -= sorted[other];
+      members[M].push_back(other);
+      load[M] += sorted[other];
+      best[other] = M;
+    }
+    members[bb].push_back(item);
+    load[bb] += sorted[item];
+    best[item] = bb;
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+// Longest-processing-time list schedule: each item (in decreasing cost) to
+// the least-loaded bin, lowest index among equals.
+std::vector<int> lpt_packing(const std::vector<double>& sorted, int P) {
+  std::vector<int> bin_of(sorted.size());
+  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>,
+                      std::greater<std::pair<double, int>>>
+      heap;
+  for (int b = 0; b < P; ++b) heap.push({0.0, b});
+  for (size_t i = 0; i < sorted.size(); ++i) {
+    auto top = heap.top();
+    heap.pop();
+    bin_of[i] = top.second;
+    heap.push({top.first + sorted[i], top.second});
+  }
+  return bin_of;
+}
+
+// Packs the n_heads tiles of each group (tile (g, h) costs gcost[g]) into P
+// bins: first-fit-decreasing under the smallest capacity that fits (found by
+// bisection), then local moves and swaps out of the fullest bin. Each bin
+// lists its tiles costliest first. False when first fit never succeeds.
+bool pack_tiles(const std::vector<double>& gcost, int n_heads, int P, TileSched& sched) {
+  const int ng = (int)gcost.size();
+  const int n_items = ng * n_heads;
+  std::vector<double> cost(n_items);
+  double total = 0.0, cmax = 0.0;
+  for (int g = 0; g < ng; ++g)
+    for (int hh = 0; hh < n_heads; ++hh) {
+      cost[g * n_heads + hh] = gcost[g];
+      total += gcost[g];
+      cmax = std::max(cmax, gcost[g]);
+    }
+  // items in decreasing cost (groups arrive in decreasing work; the modelled
+  // cost may order them slightly differently)
+  std::vector<int> order(n_items);
+  for (int i = 0; i < n_items; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return cost[x] > cost[y]; });
+  std::vector<double> sorted(n_items);
+  for (int i = 0; i < n_items; ++i) sorted[i] = cost[order[i]];
+  std::vector<int> bin_of, best;
+  double lo = std::max(cmax, total / P), hi = lo;
+  bool fits = first_fit(sorted, P, hi, best);
+  for (int tries = 0; tries < 64 && !fits; ++tries) {
+    hi *= 1.05;
+    fits = first_fit(sorted, P, hi, best);
+  }
+  if (!fits) return false;
+  for (int it = 0; it < 10; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (first_fit(sorted, P, mid, bin_of)) {
+      hi = mid;
+      best = bin_of;
+    } else {
+      lo = mid;
+    }
+  }
+  // Both first fit and LPT list scheduling, each locally improved; the
+  // better of the two (first fit wins ties). Neither start dominates.
+  {
+    std::vector<int> alt = lpt_packing(sorted, P);
+    const double m_ff = improve_packing(sorted, P, best);
+    const double m_lpt = improve_packing(sorted, P, alt);
+    if (m_lpt < m_ff) best = alt;
+  }
+  // each bin's tiles costliest first (items are in decreasing cost order)
+  std::vector<int> count(P + 1, 0);
+  for (int i = 0; i < n_items; ++i) ++count[best[i] + 1];
+  for (int b = 0; b < P; ++b) count[b + 1] += count[b];
+  for (int b = 0; b <= P; ++b) sched.bin0[b] = (uint16_t)count[b];
+  std::vector<int> fill(count.begin(), count.end() - 1);
+  for (int i = 0; i < n_items; ++i) {
+    const int item = order[i];
+    const int g = item / n_heads, hh = item % n_heads;
+    sched.tile[fill[best[i]]++] = (uint16_t)((g << 8) | hh);
+  }
+  sched.n_bins = P;
+  return true;
+}
+
+// Static schedule of the bf16 step's (group, head) tiles over the SMs, so
+// that the tiles of a persistent CTA add up to about the same modelled time
+// on every SM (list scheduling in launch order leaves the SMs that draw
+// three long tiles well behind). Cached while the group costs repeat (every
+// layer of a step shares them). n_bins = 0 asks for the one-tile kernel.
+const TileSched& tile_schedule(const std::vector<double>& gcost, int n_heads) {
+  thread_local TileSched sched;
+  thread_local std::vector<double> last_cost;
+  thread_local int last_heads = -1, last_sm = -1;
+  const int ng = (int)gcost.size();
+  const int n_items = ng * n_heads;
+  const int P = std::min(std::min(sm_count(), kMaxSchedBins), n_items);
+  // a CTA per tile already when the tiles fit on the SMs at once
+  if (ng == 0 || n_heads > 256 || ng > 256 || n_items > kMaxSchedTiles || P <= 0 ||
+      P > kMaxSchedBins || n_items <= P) {
+    sched.n_bins = 0;
+    last_heads = -1;
+    return sched;
+  }
+  if (last_heads == n_heads && last_sm == P && last_cost == gcost) return sched;
+  if (!pack_tiles(gcost, n_heads, P, sched)) {
+    sched.n_bins = 0;
+    last_heads = -1;
+    return sched;
+  }
+  last_cost = gcost;
+  last_heads = n_heads;
+  last_sm = P;
+  return sched;
 }
 
 }  // namespace
@@ -336,6 +537,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   plan.layer = layer;
   for (int b = 0; b <= st->batch; ++b) plan.cu_rows[b] = st->cu_rows[b];
   for (int b = 0; b < st->batch; ++b) plan.seq_lens[b] = st->seq_lens[b];
+  std::vector<double> gcost;   // modelled tile duration of each group
   // Row groups (one 128-row tile each): whole sequences, each padded to a
   // multiple of 16 q rows (the attention MMA's N granularity), packed first
   // fit in order of decreasing size. The bf16 kernel also keeps a group's
@@ -351,6 +553,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
       long long cost;
       std::vector<int> seqs;
     };
+    gcost.clear();
     std::vector<int> idx;
     for (int b = 0; b < st->batch; ++b) {
       plan.seq_qoff[b] = 0;
@@ -404,6 +607,21 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
     }
     plan.group_seq0[groups.size()] = k;
     plan.n_groups = (int)groups.size();
+    // Modelled duration of a group's tile on B200 (us, fitted to measured
+    // tile timelines): the projection grows with the number of x boxes (one
+    // per power-of-two piece of each sequence's padded rows), attention
+    // with the 128-key chunks, a little more for wider sequences.
+    for (const Grp& gp : groups) {
+      int nbox = 0;
+      double attn = 0.0;
+      for (int b : gp.seqs) {
+        nbox += __builtin_popcount((unsigned)(n16(b) / 16));
+        const int ctx = (st->seq_lens[b] + c.page_size - 1) / c.page_size;
+        const int extra = (rows_of(b) + c.page_size - 1) / c.page_size + 1;
+        attn += 0.53 + ((ctx + extra + 1) / 2) * (2.58 + 0.144 * (n16(b) / 16));
+      }
+      gcost.push_back(46.9 + 2.93 * nbox + attn);
+    }
   }
   const int ng = plan.n_groups;
 
@@ -441,7 +659,8 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
       }
       if (!encode_wqkv_5d(&tw, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim))
         return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv)");
-      e = launch_step_bf16(plan, a, txp, &tw, &h->tmap_k, &h->tmap_v, s);
+      e = launch_step_bf16(plan, tile_schedule(gcost, c.n_heads), a, txp, &tw, &h->tmap_k,
+                           &h->tmap_v, s);
     } else {
       e = launch_step_f32(plan, a, s);
     }
@@ -498,6 +717,31 @@ fdllm_status fdllm_verify_accept(const void* mask_logits, int32_t dtype, int32_t
                                        reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "verify_accept: launch");
   g_last_launches = rows > 0 ? 2 : 1;
+  return FDLLM_OK;
+}
+
+fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_t n_groups,
+                                      int32_t n_heads, int32_t n_bins, int32_t* bin_start,
+                                      int32_t* tiles) {
+  if (!group_cost || !bin_start || !tiles)
+    return fail(FDLLM_ERR_INVALID_ARG, "plan_tile_schedule: null pointer");
+  if (n_groups <= 0 || n_heads <= 0 || n_bins <= 0)
+    return fail(FDLLM_ERR_INVALID_ARG, "plan_tile_schedule: sizes must be positive");
+  if (n_groups > 256 || n_heads > 256 || n_groups * n_heads > kMaxSchedTiles ||
+      n_bins > kMaxSchedBins)
+    return fail(FDLLM_ERR_UNSUPPORTED,
+                "plan_tile_schedule: at most 256 groups, 256 heads, %d tiles and %d bins",
+                kMaxSchedTiles, kMaxSchedBins);
+  std::vector<double> gc(group_cost, group_cost + n_groups);
+  for (double v : gc)
+    if (!(v >= 0.0) || !std::isfinite(v))
+      return fail(FDLLM_ERR_INVALID_ARG, "plan_tile_schedule: costs must be finite and >= 0");
+  TileSched ts;
+  if (!pack_tiles(gc, n_heads, n_bins, ts))
+    return fail(FDLLM_ERR_UNSUPPORTED, "plan_tile_schedule: no packing found");
+  for (int b = 0; b <= n_bins; ++b) bin_start[b] = ts.bin0[b];
+  for (int i = 0; i < n_groups * n_heads; ++i)
+    tiles[i] = (ts.tile[i] >> 8) * n_heads + (ts.tile[i] & 255);
   return FDLLM_OK;
 }
 

@@ -39,6 +39,19 @@ struct StepPlan {
                                    // (a multiple of 16)
 };
 
+// Static tile schedule of the bf16 step: CTA i runs tiles
+// tile[bin0[i] .. bin0[i+1]) in order, each encoded g << 8 | h. With
+// n_bins == 0 the one-tile kernel runs instead, CTA i on tile i (group-major
+// order). The schedule travels as a kernel parameter, so it is kept small
+// (a larger parameter block costs launch time).
+constexpr int kMaxSchedTiles = 1024;
+constexpr int kMaxSchedBins = 160;
+struct TileSched {
+  int n_bins;
+  uint16_t bin0[kMaxSchedBins + 1];
+  uint16_t tile[kMaxSchedTiles];
+};
+
 // Per-call device pointers and pool geometry.
 struct StepArgs {
   const void* x;
@@ -64,9 +77,9 @@ struct StepArgs {
 
 // Launchers (return cudaGetLastError()).
 // tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
-cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* const* tmap_x,
-                             const void* tmap_w, const void* tmap_k, const void* tmap_v,
-                             cudaStream_t stream);
+cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
+                             const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                             const void* tmap_v, cudaStream_t stream);
 cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
                                cudaStream_t stream);

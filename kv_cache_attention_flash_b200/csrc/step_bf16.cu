@@ -38,6 +38,7 @@
 #include <cuda_bf16.h>
 
 #include <cstddef>
+#include <type_traits>
 
 #include "fdllm_internal.h"
 #include "ptx.cuh"
@@ -225,8 +226,18 @@ __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool
   }
 }
 
+// Schedule parameter of the one-tile kernel: none.
+struct NoSched {
+  int n_bins;
+};
+
+// kPersist: a persistent CTA runs the tiles of its schedule bin; otherwise
+// CTA i runs tile i.
+template <bool kPersist>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    step_bf16_kernel(const __grid_constant__ StepPlan plan, const __grid_constant__ StepArgs a,
+    step_bf16_kernel(const __grid_constant__ StepPlan plan,
+                     const __grid_constant__ std::conditional_t<kPersist, TileSched, NoSched> sched,
+                     const __grid_constant__ StepArgs a,
                      const __grid_constant__ CUtensorMap tmap_x16,
                      const __grid_constant__ CUtensorMap tmap_x32,
                      const __grid_constant__ CUtensorMap tmap_x64,
@@ -242,14 +253,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  // tiles are numbered group-major (groups in order of decreasing work)
-  const int g = blockIdx.x / a.n_heads;
-  const int h = blockIdx.x % a.n_heads;
-  // sequences of this group: plan.seq_order[seq_a .. seq_b); sequence b
-  // owns q rows [seq_qoff[b], seq_qoff[b] + n_b) of the 128-row tile, which
-  // are also the TMEM lanes of the projection
-  const int seq_a = plan.group_seq0[g];
-  const int seq_b = plan.group_seq0[g + 1];
   const int H = a.hidden;
   const int nkb = H / BK;
   const int layer = plan.layer;
@@ -293,6 +296,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
 
+  // Tiles of this CTA (a persistent CTA runs several, one after another;
+  // barrier phases, schedule counters and TMEM carry over between them).
+  int t_beg = 0, t_end = 1;
+  if constexpr (kPersist) {
+    t_beg = sched.bin0[blockIdx.x];
+    t_end = sched.bin0[blockIdx.x + 1];
+  }
+  uint32_t kstep0 = 0;   // projection K steps of the earlier tiles
+  // attention schedule counters, identical in every thread: chunk loads (K
+  // or V) issued so far, S^T products, P.V products, finished sequences and
+  // sequences whose q rows were repeated
+  uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0, qcount = 0;
+  for (int ti = t_beg; ti < t_end; ++ti) {
+  int g, h;
+  if constexpr (kPersist) {
+    g = sched.tile[ti] >> 8;
+    h = sched.tile[ti] & 255;
+  } else {   // group-major numbering (groups in order of decreasing work)
+    g = blockIdx.x / a.n_heads;
+    h = blockIdx.x % a.n_heads;
+  }
+  // sequences of this group: plan.seq_order[seq_a .. seq_b); sequence b
+  // owns q rows [seq_qoff[b], seq_qoff[b] + n_b) of the 128-row tile, which
+  // are also the TMEM lanes of the projection
+  const int seq_a = plan.group_seq0[g];
+  const int seq_b = plan.group_seq0[g + 1];
+
   // ================================================================ projection
   if (warp == kProducerWarp) {
     if (lane == 0) {   // TMA producer
@@ -317,8 +347,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const int u = kb / STAGES;
+        const uint32_t kg = kstep0 + kb;
+        const int s = kg % STAGES;
+        const uint32_t u = kg / STAGES;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
         uint8_t* st = smem + s * STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&ctrl->full[s], B_BYTES + x_rows * BK * 2);
@@ -341,8 +372,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, 128, false, true);
       constexpr uint32_t idesc256 = ptx::idesc_bf16_f32(BM, 256, false, true);
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES;
-        const int u = kb / STAGES;
+        const uint32_t kg = kstep0 + kb;
+        const int s = kg % STAGES;
+        const uint32_t u = kg / STAGES;
         if (!wait_bar(ctrl, &ctrl->full[s], u & 1, a.err, 2)) break;
         ptx::tc_fence_after();
         const uint32_t a_base = ptx::smem_u32(smem + s * STAGE_BYTES);
@@ -579,10 +611,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t slot_base = ptx::smem_u32(smem + SLOT_OFF);
   const uint32_t pt_base = ptx::smem_u32(smem + PT_OFF);
   const uint32_t qrep_base = ptx::smem_u32(smem + QREP_OFF);
-  // Schedule counters, identical in every thread: chunk loads (K or V)
-  // issued so far, S^T products, P.V products, finished sequences and
-  // sequences whose q rows were repeated.
-  uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0, qcount = 0;
 
   const int nseq_g = ctrl->nseq;
   for (int si = 0; si < nseq_g; ++si) {
@@ -1009,46 +1037,67 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!wide) ++qcount;
   }
 
-  // ================================================================ teardown
+  // ================================================================ tile end
+  // Before the next tile's projection reuses shared memory and TMEM, and
+  // before TMEM is freed: every tcgen05 operation of this tile has completed
+  // (the second completion of mma_done in the tile) and the last chunk loads
+  // have landed (they have, unless a wait timed out).
   if (warp == kMmaWarp && lane == 0) {
-    // every tcgen05 operation issued by this thread has completed
     ptx::umma_commit(&ctrl->mma_done);
     ptx::mbar_wait(&ctrl->mma_done, 1, WAIT_NS);
   }
   if (warp == kProducerWarp && lane == 0 && ring > 0) {
-    // the last chunk loads have landed (they have, unless a wait timed out)
     for (uint32_t it = ring > NSLOT ? ring - NSLOT : 0; it < ring; ++it)
       ptx::mbar_wait(&ctrl->afull[it % NSLOT], (it / NSLOT) & 1, WAIT_NS);
   }
   __syncwarp();
+  if constexpr (kPersist) {
+    fence_async_smem();   // st.shared of this tile before the next tile's TMA writes
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    kstep0 += nkb;
+  }
+  }   // tiles
+
+  // ================================================================ teardown
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, TMEM_COLS);
+}
+
+template <bool kPersist, typename Sched>
+cudaError_t launch_kernel(int grid, const StepPlan& plan, const Sched& sched, const StepArgs& a,
+                          const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                          const void* tmap_v, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(step_bf16_kernel<kPersist>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  step_bf16_kernel<kPersist><<<grid, NTHREADS, SMEM_BYTES, stream>>>(
+      plan, sched, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
+      *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
+      *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
+      *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_k),
+      *reinterpret_cast<const CUtensorMap*>(tmap_v));
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t step_bf16_smem_bytes() { return SMEM_BYTES; }
 
-cudaError_t launch_step_bf16(const StepPlan& plan, const StepArgs& a, const void* const* tmap_x,
-                             const void* tmap_w, const void* tmap_k, const void* tmap_v,
-                             cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(step_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
+                             const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                             const void* tmap_v, cudaStream_t stream) {
+  if (sched.n_bins > 0)
+    return launch_kernel<true>(sched.n_bins, plan, sched, a, tmap_x, tmap_w, tmap_k, tmap_v, stream);
   const int grid = plan.n_groups * a.n_heads;
   if (grid == 0) return cudaSuccess;
-  step_bf16_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(
-      plan, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_k),
-      *reinterpret_cast<const CUtensorMap*>(tmap_v));
-  return cudaGetLastError();
+  return launch_kernel<false>(grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_k, tmap_v, stream);
 }
 
 }  // namespace fdllm
