@@ -75,7 +75,9 @@ def captured_traffic(name: str):
     if traffic is None or want is None:
         return None
     csrc = os.path.join(ROOT, "kv_cache_attention_flash_b200", "csrc")
-    have = [code_hash(os.path.join(csrc, f)) for f in ("step_bf16.cu", "ptx.cuh")]
+    # the kernel, its PTX helpers and the host code that plans its launch
+    # (row groups and the tile schedule decide what each CTA reads)
+    have = [code_hash(os.path.join(csrc, f)) for f in ("step_bf16.cu", "ptx.cuh", "api.cu")]
     return traffic if have == want else None
 
 
