@@ -78,9 +78,61 @@ constexpr int SEL_MAXK = 1024;
 constexpr int SEL_MAXL = 65536;
 constexpr int SEL_SMEM_KEYS = 5120;   // rows up to this length keep their keys on chip
 
-// One CTA per sequence. Exact radix select of the k-th largest key (4 passes
-// of 8 bits), then the strictly larger keys plus the lowest-slot ties, then a
-// bitonic sort by (key descending, slot ascending).
+// A candidate as one 64-bit word ordered like (key descending, slot
+// ascending): key in the high half, the slot's complement in the low half.
+// 0 marks "no candidate" (below every real one: slots are < 2^31).
+__device__ __forceinline__ uint64_t cand_word(uint32_t key, int slot) {
+  return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)slot);
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Bitonic sort across a warp, one word per lane: lane i ends with the i-th
+// largest. Blocks of `size` lanes alternate direction until the last stage.
+__device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t o = shfl_xor_u64(v, stride);
+      const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+      v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  return v;
+}
+
+// The 32 largest of two descending warp lists: the elementwise maximum of
+// one list and the other reversed is bitonic and holds them; a bitonic merge
+// sorts it.
+__device__ __forceinline__ uint64_t warp_merge_top(uint64_t a, uint64_t b, int lane) {
+  const uint64_t br = shfl_u64(b, 31 - lane);
+  uint64_t c = a > br ? a : br;
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t o = shfl_xor_u64(c, stride);
+    c = (lane & stride) == 0 ? (c > o ? c : o) : (c < o ? c : o);
+  }
+  return c;
+}
+
+// One CTA per sequence.
+// k <= 32: each warp keeps the 32 largest candidate words of its chunks of
+// 32 slots, sorted in registers (a chunk is sorted only when one of its
+// words beats the warp's 32nd); the warps' lists are then merged pairwise.
+// Larger k: exact radix select of the k-th largest key (4 passes of 8 bits),
+// then the strictly larger keys plus the lowest-slot ties, then a bitonic
+// sort by (key descending, slot ascending). Both give the same slots in the
+// same order.
 __global__ void __launch_bounds__(SEL_THREADS)
     select_kernel(const float* mass, const int32_t* seq_lens, int row_stride, int k,
                   const int32_t* exclude_cu, const int32_t* exclude_slots, int32_t* tracked) {
@@ -101,8 +153,10 @@ __global__ void __launch_bounds__(SEL_THREADS)
   __shared__ uint32_t sk[SEL_MAXK];
   __shared__ int ss[SEL_MAXK];
   __shared__ int warp_sums[SEL_THREADS / 32];
-  __shared__ uint32_t skey[SEL_SMEM_KEYS];
-  const bool staged = L <= SEL_SMEM_KEYS;
+  __shared__ __align__(16) uint32_t skey[SEL_SMEM_KEYS];
+  static_assert(SEL_THREADS * 8 <= SEL_SMEM_KEYS * 4, "warp lists fit in the key buffer");
+  const bool fast = k <= 32;
+  const bool staged = !fast && L <= SEL_SMEM_KEYS;
   if (staged)
     for (int j = tid; j < L; j += SEL_THREADS) skey[j] = fkey(__ldg(m + j));
   auto key_of = [&](int j) -> uint32_t { return staged ? skey[j] : fkey(__ldg(m + j)); };
@@ -118,6 +172,35 @@ __global__ void __launch_bounds__(SEL_THREADS)
   }
   if (tid == 0) s_total = 0;
   __syncthreads();
+  if (fast) {
+    constexpr int NW = SEL_THREADS / 32;
+    const int lane = tid & 31, warp = tid >> 5;
+    uint64_t top = 0;
+    for (int base = warp * 32; base < L; base += SEL_THREADS) {
+      const int j = base + lane;
+      uint64_t v = 0;
+      if (j < L && !((excl[j >> 5] >> (j & 31)) & 1u)) v = cand_word(fkey(__ldg(m + j)), j);
+      if (__ballot_sync(0xffffffffu, v > shfl_u64(top, 31)) == 0u) continue;
+      top = warp_merge_top(top, warp_sort_desc(v, lane), lane);
+    }
+    uint64_t* lists = reinterpret_cast<uint64_t*>(skey);   // [NW][32], unused in this path
+    lists[warp * 32 + lane] = top;
+    __syncthreads();
+#pragma unroll 1
+    for (int half = NW / 2; half > 0; half >>= 1) {
+      if (warp < half) {
+        const uint64_t c = warp_merge_top(lists[warp * 32 + lane], lists[(warp + half) * 32 + lane],
+                                          lane);
+        lists[warp * 32 + lane] = c;
+      }
+      __syncthreads();
+    }
+    if (tid < k) {
+      const uint64_t c = lists[tid];
+      tracked[(size_t)b * k + tid] = c ? (int)(0xFFFFFFFFu - (uint32_t)c) : -1;
+    }
+    return;
+  }
   // candidate count (one shared atomic per warp)
   {
     int c = 0;

@@ -147,19 +147,22 @@ def test_two_views_isolated_bitwise_on_gpu():
 
 
 def test_select_tracked_matches_oracle_exactly():
+    # k <= 32 takes the warp-list path, larger k the radix-select path
     rng = np.random.default_rng(7)
-    for trial in range(12):
+    for trial in range(24):
         B = int(rng.integers(1, 9))
-        stride = int(rng.choice([64, 300, 1024, 4096, 9000]))
-        k = int(rng.choice([1, 8, 32, 64, 200, 1024]))
+        stride = int(rng.choice([64, 300, 1024, 4096, 9000, 20000]))
+        k = int(rng.choice([1, 8, 31, 32, 33, 64, 200, 1024]))
         lens = rng.integers(0, stride + 1, B).astype(np.int32)
         # many exact ties: values on a coarse grid
         mass = (rng.integers(0, 50, (B, stride)) / 997.0).astype(np.float32)
         if trial % 2:
             mass = rng.random((B, stride)).astype(np.float32)
-        if trial == 10:      # every key equal: the k lowest slots, in order
+        if trial in (10, 22):      # every key equal: the k lowest slots, in order
+            k = 200 if trial == 10 else 32
             mass = np.full((B, stride), 1e-3, np.float32)
-        if trial == 11:      # mostly zeros, a few distinct values on top
+        if trial in (11, 23):      # mostly zeros, a few distinct values on top
+            k = 64 if trial == 11 else 16
             mass = np.zeros((B, stride), np.float32)
             mass[:, ::97] = rng.random((B, len(range(0, stride, 97)))).astype(np.float32)
         ex = [rng.choice(max(int(L), 1), size=min(int(L), 5), replace=False) if L else np.zeros(0, int) for L in lens]
