@@ -226,6 +226,29 @@ __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool
   }
 }
 
+// Running log2-domain max m and sum l of one row over NK more scores v
+// (raw S values; the scale sl2 = log2(e)/sqrt(D) is applied in the
+// exponent's FMA). Keys whose bit in mk is clear are dropped before
+// anything else, so a NaN in an unattended slot never reaches the sums.
+// Four independent max / sum chains.
+template <int NK>
+__device__ __forceinline__ void lse_block(float* v, uint32_t mk, float sl2, float& m, float& l) {
+  float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int j = 0; j < NK; ++j) {
+    v[j] = ((mk >> j) & 1u) ? v[j] : -INFINITY;
+    b4[j & 3] = fmaxf(b4[j & 3], v[j]);
+  }
+  // rounding is monotone, so the scaled maximum is the maximum scaled score
+  const float mn = fmaxf(m, fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3])) * sl2);
+  if (mn == -INFINITY) return;
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < NK; ++j) s4[j & 3] += ptx::ex2(fmaf(v[j], sl2, -mn));
+  l = l * ptx::ex2(m - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  m = mn;
+}
+
 // Schedule parameter of the one-tile kernel: none.
 struct NoSched {
   int n_bins;
@@ -871,35 +894,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                   }
                 }
               }
-              uint32_t mk = active ? (uint32_t)(km >> (j0 & 63)) : 0u;
-              if (nk < 32) mk &= (1u << nk) - 1u;
+              const uint32_t mk = active ? (uint32_t)(km >> (j0 & 63)) : 0u;
               float v[32];
               const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + j0;
               if (nk == 32) {
                 ptx::tmem_ld32(sbase, v);
+                ptx::tmem_ld_wait();
+                lse_block<32>(v, mk, sl2, m, l);
               } else {
                 ptx::tmem_ld16(sbase, v);
-#pragma unroll
-                for (int j = 16; j < 32; ++j) v[j] = -INFINITY;
-              }
-              ptx::tmem_ld_wait();
-              // four independent max / sum chains
-              float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                v[j] *= sl2;
-                b4[j & 3] = fmaxf(b4[j & 3], ((mk >> j) & 1u) ? v[j] : -INFINITY);
-              }
-              const float mn = fmaxf(m, fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3])));
-              if (mn != -INFINITY) {
-                float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                  const float e = ptx::ex2(v[j] - mn);
-                  s4[j & 3] += ((mk >> j) & 1u) ? e : 0.f;
-                }
-                l = l * ptx::ex2(m - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-                m = mn;
+                ptx::tmem_ld_wait();
+                lse_block<16>(v, mk, sl2, m, l);
               }
             }
           }
