@@ -298,46 +298,104 @@ def e2e_measure(wl: Workload, steps: int):
     """Same metric through the public API with host buffers: per step the
     inputs (x of every layer, positions, slots, views, block table) are copied
     from pinned host memory, and out, attn_mass and the tracked set are read
-    back; all inside the timed region."""
-    fd = wl.fd
-    dev = wl.device
-    hx = [x.cpu().pin_memory() for x in wl.x]
-    hpos = wl.pos.cpu().pin_memory()
-    hslots = wl.slots.cpu().pin_memory()
-    hview = wl.view.cpu().pin_memory()
-    hbt = wl.bt.cpu().pin_memory()
-    dx = [torch.empty_like(x) for x in wl.x]
-    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    hmass = torch.empty(wl.mass.shape, dtype=wl.mass.dtype).pin_memory()
-    htr = torch.empty(wl.tracked.shape, dtype=wl.tracked.dtype).pin_memory()
-    h2d = sum(x.numel() * x.element_size() for x in hx) + sum(
-        t.numel() * t.element_size() for t in (hpos, hslots, hview, hbt))
-    d2h = sum(t.numel() * t.element_size() for t in (hout, hmass, htr))
+    back; all inside the timed region.
 
-    def one():
+    Returns (pipelined ms, serial ms, h2d bytes, d2h bytes) per step.
+    Serial: copy in, compute and copy out one after another on one stream.
+    Pipelined, as a serving loop runs it: uploads on one stream and
+    downloads on another, with device and host buffers doubled, so that step
+    i+1's inputs go up and step i-1's outputs come down while step i
+    computes. Every step still moves all of its bytes inside the timed
+    region."""
+    fd = wl.fd
+    m = wl.meta
+    NB = 2
+    hx = [x.cpu().pin_memory() for x in wl.x]
+    dmeta0 = (wl.pos, wl.slots, wl.view, wl.bt)
+    hmeta = [t.cpu().pin_memory() for t in dmeta0]
+    bufs = []
+    for _ in range(NB):
+        bufs.append({
+            "x": [torch.empty_like(x) for x in wl.x],
+            "meta": [torch.empty_like(t) for t in dmeta0],
+            "out": torch.empty_like(wl.out), "mass": torch.empty_like(wl.mass),
+            "tr": torch.empty_like(wl.tracked),
+            "hout": torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory(),
+            "hmass": torch.empty(wl.mass.shape, dtype=wl.mass.dtype).pin_memory(),
+            "htr": torch.empty(wl.tracked.shape, dtype=wl.tracked.dtype).pin_memory(),
+            "ev_in": torch.cuda.Event(), "ev_comp": torch.cuda.Event(), "ev_out": torch.cuda.Event(),
+        })
+    h2d = sum(x.numel() * x.element_size() for x in hx) + sum(
+        t.numel() * t.element_size() for t in hmeta)
+    d2h = sum(t.numel() * t.element_size() for t in (bufs[0]["hout"], bufs[0]["hmass"],
+                                                      bufs[0]["htr"]))
+    comp = torch.cuda.current_stream()
+    s_in = torch.cuda.Stream()
+    s_out = torch.cuda.Stream()
+
+    def compute(b, stream):
+        pos, slots, view, bt = b["meta"]
         for l in range(wl.n_layers):
-            dx[l].copy_(hx[l], non_blocking=True)
-        wl.pos.copy_(hpos, non_blocking=True)
-        wl.slots.copy_(hslots, non_blocking=True)
-        wl.view.copy_(hview, non_blocking=True)
-        wl.bt.copy_(hbt, non_blocking=True)
-        wl.step(x_list=dx)
-        hout.copy_(wl.out, non_blocking=True)
-        hmass.copy_(wl.mass, non_blocking=True)
-        htr.copy_(wl.tracked, non_blocking=True)
+            fd.fdllm_layer_step(wl.cache.handle, l, m.cu_rows, m.seq_lens, m.max_blocks, b["x"][l],
+                                wl.w[l], pos, bt, view, b["out"], b["mass"], slots, stream=stream)
+        fd.fdllm_select_tracked(b["mass"], wl.seq_lens_d, m.track_k, wl.ex_cu, wl.ex_sl, b["tr"],
+                                stream=stream)
+
+    def one_serial():
+        b = bufs[0]
+        for l in range(wl.n_layers):
+            b["x"][l].copy_(hx[l], non_blocking=True)
+        for d, h in zip(b["meta"], hmeta):
+            d.copy_(h, non_blocking=True)
+        compute(b, comp)
+        b["hout"].copy_(b["out"], non_blocking=True)
+        b["hmass"].copy_(b["mass"], non_blocking=True)
+        b["htr"].copy_(b["tr"], non_blocking=True)
+
+    def one_pipelined(i):
+        b = bufs[i % NB]
+        if i >= NB:   # step i-NB no longer reads these inputs
+            s_in.wait_event(b["ev_comp"])
+        with torch.cuda.stream(s_in):
+            for l in range(wl.n_layers):
+                b["x"][l].copy_(hx[l], non_blocking=True)
+            for d, h in zip(b["meta"], hmeta):
+                d.copy_(h, non_blocking=True)
+            b["ev_in"].record(s_in)
+        comp.wait_event(b["ev_in"])
+        if i >= NB:   # step i-NB's outputs have come down
+            comp.wait_event(b["ev_out"])
+        compute(b, comp)
+        b["ev_comp"].record(comp)
+        s_out.wait_event(b["ev_comp"])
+        with torch.cuda.stream(s_out):
+            b["hout"].copy_(b["out"], non_blocking=True)
+            b["hmass"].copy_(b["mass"], non_blocking=True)
+            b["htr"].copy_(b["tr"], non_blocking=True)
+            b["ev_out"].record(s_out)
+
+    def timed(run):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(steps):
+            run(i)
+        comp.wait_stream(s_in)
+        comp.wait_stream(s_out)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
 
     for _ in range(3):
-        one()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(steps):
-        one()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    return ms, h2d, d2h
+        one_serial()
+    serial_ms = timed(lambda i: one_serial())
+    for i in range(3):
+        one_pipelined(i)
+    pipe_ms = timed(one_pipelined)
+    return pipe_ms, serial_ms, h2d, d2h
 
 
 # ------------------------------------------------------------------ main arms
@@ -447,11 +505,10 @@ def run_native(args):
             "hbm_gbs_achieved": byt / kern_s / 1e9,
             "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline": max(t_hbm, t_tc) / kern_s}
 
-    e2e_ms, h2d, d2h = e2e_measure(wl, max(10, min(args.steps, 200)))
-    e2e_val_local = meta.total_rows / (e2e_ms / 1000.0)
+    e2e_ms, serial_ms, h2d, d2h = e2e_measure(wl, max(10, min(args.steps, 200)))
     e2e_ms_max = reduce_max(e2e_ms, dev)
+    serial_ms_max = reduce_max(serial_ms, dev)
     e2e_value = meta.total_rows * world / (e2e_ms_max / 1000.0)
-    del e2e_val_local
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -467,7 +524,9 @@ def run_native(args):
         "layer_steps_per_s": value / meta.total_rows * spec.shape.n_layers,
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms_max},
+                "ms_per_step": e2e_ms_max, "copies": "pipelined (upload, compute, download streams)",
+                "serial_value": meta.total_rows * world / (serial_ms_max / 1000.0),
+                "serial_ms_per_step": serial_ms_max},
         "gpu_launches": launches, "clocks": clocks,
     }
     if rank == 0:
