@@ -369,6 +369,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           rem -= hgt;
         }
       }
+      // x rows are read by every head's tile of the group and a head's
+      // Wqkv slice by every group's tile: keep both in L2
+      const uint64_t pol_keep = ptx::policy_evict_last();
       for (int kb = 0; kb < nkb; ++kb) {
         const uint32_t kg = kstep0 + kb;
         const int s = kg % STAGES;
@@ -381,13 +384,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (i < nbox) {
             const CUtensorMap* mx = box_h[i] == 128 ? &tmap_x128 : box_h[i] == 64 ? &tmap_x64
                                   : box_h[i] == 32 ? &tmap_x32 : &tmap_x16;
-            ptx::tma_load_2d(st + box_dst[i], mx, kb * BK, box_row[i], &ctrl->full[s]);
+            ptx::tma_load_2d_hint(st + box_dst[i], mx, kb * BK, box_row[i], &ctrl->full[s],
+                                  pol_keep);
           }
         }
         // this head's q, k and v column blocks of Wqkv, two 64-column halves
         // each: one 48 KB box of the 5-D view (column, K row, half, block,
         // head), laid out as six [64 K rows][64 columns] sub-boxes
-        ptx::tma_load_5d(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s]);
+        ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
+                              pol_keep);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -680,7 +685,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------- TMA producer
       if (lane == 0) {
         uint32_t item = r0;
-        auto load = [&](int c, bool is_v) {
+        // pass-1 K chunks come back for pass 2 a few chunks later: keep
+        // them in L2; pass-2 K and V are read for the last time
+        const uint64_t pol_keep = ptx::policy_evict_last();
+        const uint64_t pol_drop = ptx::policy_evict_first();
+        auto load = [&](int c, bool is_v, uint64_t pol) {
           const int s = item % NSLOT;
           const uint32_t u = item / NSLOT;
           if (u > 0) wait_bar(ctrl, &ctrl->aempty[s], (u - 1) & 1, a.err, 10);
@@ -699,16 +708,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int pi = 0; pi < 2; ++pi) {
             if (phys[pi] < 0) continue;
             const int row = ((layer * a.num_pages + phys[pi]) * a.n_heads + h) * PS;
-            ptx::tma_load_2d(dst + pi * BOX_BYTES, map, 0, row, &ctrl->afull[s]);
-            ptx::tma_load_2d(dst + HALF_BYTES + pi * BOX_BYTES, map, 64, row, &ctrl->afull[s]);
+            ptx::tma_load_2d_hint(dst + pi * BOX_BYTES, map, 0, row, &ctrl->afull[s], pol);
+            ptx::tma_load_2d_hint(dst + HALF_BYTES + pi * BOX_BYTES, map, 64, row, &ctrl->afull[s],
+                                  pol);
           }
           ++item;
         };
-        for (int c = 0; c < nch; ++c) load(c, false);
-        for (int c = 0; c < npre; ++c) load(c, false);
+        for (int c = 0; c < nch; ++c) load(c, false, pol_keep);
+        for (int c = 0; c < npre; ++c) load(c, false, pol_drop);
         for (int c = 0; c < nch; ++c) {
-          load(c, true);
-          if (c + 2 < nch) load(c + 2, false);
+          load(c, true, pol_drop);
+          if (c + 2 < nch) load(c + 2, false, pol_drop);
         }
       }
     } else if (warp == kMmaWarp) {
