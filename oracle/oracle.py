@@ -32,8 +32,9 @@ Readings where the pages are silent (each is listed in the design notes):
     (lowest id among equal logits) is the drafted token; the confidence is
     that token's softmax probability; the threshold is a parameter.
 
-Every function here has a pin in tests/test_oracle_pins.py (brute force,
-closed forms, library special cases or invariants); none is "parity
+Every function here has a pin in tests/test_oracle_pins.py,
+tests/test_oracle_verify_pins.py or tests/test_oracle_oproj_pins.py (brute
+force, closed forms, library special cases or invariants); none is "parity
 unpinned".
 """
 from __future__ import annotations
@@ -308,3 +309,23 @@ def verify_accept(pred, conf, draft_tokens, cu_rows, tau: float):
                 break
         out[b] = n
     return out
+
+
+# --------------------------------------------------------------------------
+# Output projection of the attention block (a "next" step after the layer)
+# --------------------------------------------------------------------------
+
+def oproj(out_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
+    """The attention block's output projection y = o W_o, float64.
+
+    o [R, H] holds each row's attention output with the heads side by side
+    (head h in columns h*D .. h*D + D - 1, the layout of the layer step's
+    `out`), given as bf16 bits; W_o [H, H] is row-major bf16 bits, no bias.
+    The pages stop at the attention output ([FD ¶1]: QKV projection, RoPE,
+    cache write, scheduled attention) and say nothing of W_o; this is the
+    plain linear map that follows attention in a transformer layer, read
+    with the same conventions as Wqkv (y = x W, row-major, no bias).
+    Returns float64 [R, H]; rounding y to bf16 is the caller's business."""
+    o = bf16_bits_to_f64(out_bits)
+    w = bf16_bits_to_f64(w_bits)
+    return o @ w
