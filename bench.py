@@ -5,6 +5,8 @@
 `--workload verify_b8` measures the Flash-Verify acceptance step instead
 (mask-view logits of 8 x 32 block positions over the 126464-token LLaDA
 vocabulary, bf16): positions/s, HBM roofline of the logits read.
+`--workload oproj_b32` measures the output projection y = o W_o of the
+batch-32 step's 1536 rows at hidden 4096 (bf16): rows/s, tensor roofline.
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 the fused layer step (projection, RoPE, cache write, scheduled attention,
@@ -710,13 +712,170 @@ def run_verify(args):
     return 0
 
 
+OPROJ_METRIC = "output projection rows/s; achieved TFLOP/s and % of roofline (1\u00d7B200)"
+OPROJ_UNIT = "rows/s"
+
+
+def oproj_oracle_sample(o_cpu, w_cpu, budget_s):
+    """The oracle's y = o W_o on whole row blocks of 64 until the budget."""
+    from oracle import oracle as O
+    ob, wb = W.bits_np(o_cpu), W.bits_np(w_cpu)
+    rows = 0
+    t0 = time.perf_counter()
+    while rows < ob.shape[0] and time.perf_counter() - t0 < budget_s:
+        O.oproj(ob[rows:rows + 64], wb)
+        rows += min(64, ob.shape[0] - rows)
+    dt = time.perf_counter() - t0
+    desc = (f"oracle (numpy float64 matmul) on {rows} of {ob.shape[0]} rows x "
+            f"{ob.shape[1]} x {wb.shape[1]}, 64 rows per call, {dt:.1f} s")
+    return rows / dt, desc
+
+
+def oproj_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_oproj(args):
+    """The output projection y = o W_o alone: one tcgen05 GEMM per step."""
+    rank, world, local = dist_env()
+    spec = W.OPROJ_WORKLOADS[args.workload]
+    R, H = spec.rows, spec.hidden
+    config = {"workload": spec.name, "rows": R, "hidden": H, "operands": "bf16 in, bf16 out",
+              "l2": "flushed between timed steps (256 MB write)",
+              "parallelism": f"replicas x{world}", "seed": args.seed}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        o, w = W.make_oproj(spec, args.seed)
+        budget = max(2.0, 20.0 / max(1, args.steps + args.warmup))
+        vals, desc = [], ""
+        for i in range(args.warmup + args.steps):
+            v, desc = oproj_oracle_sample(o, w, budget)
+            if i >= args.warmup:
+                vals.append(v)
+        value = float(np.mean(vals))
+        print(json.dumps({
+            "impl": "reference", "metric": OPROJ_METRIC, "value": value, "unit": OPROJ_UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * R / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": value, "unit": OPROJ_UNIT, "cores": oproj_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": OPROJ_UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}))
+        return 0
+    import kv_cache_attention_flash_b200 as fd
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    o, w = W.make_oproj(spec, args.seed + rank, device=dev)
+    y = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        fd.fdllm_oproj(o, w, y)
+        return fd.fdllm_last_launch_count()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches = 0
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev_s[i].record()
+        launches += step()
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    if sampler:
+        sampler.mark(t_wall0, t_wall1)
+        time.sleep(0.25)
+        sampler.stop()
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    total_ms, _, value = aggregate(float(sum(step_ms)), R * args.steps, dev)
+    kern_s = float(np.mean(step_ms)) / 1000.0
+    fl = 2.0 * R * H * H
+    byt = 2.0 * (R * H + H * H + R * H)
+    achieved = fl / kern_s / 1e12
+    peak = peaks["bf16_tflops"]
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": None, "peak_source": f"{peak_src} (burst)",
+            "kernel": "fdllm_oproj (tcgen05 GEMM)", "kernel_us": kern_s * 1e6,
+            "algorithmic_flops": fl, "algorithmic_bytes": byt,
+            "hbm_gbs_achieved": byt / kern_s / 1e9,
+            "roofline_us": max(byt / (peaks["hbm_gbs"] * 1e9), fl / (peak * 1e12)) * 1e6}
+    # end to end: o up from pinned host memory, y down, every step
+    ho = o.cpu().pin_memory()
+    hy = torch.empty(R, H, dtype=torch.bfloat16).pin_memory()
+    do = torch.empty_like(o)
+    n_e2e = max(10, min(args.steps, 200))
+
+    def one():
+        do.copy_(ho, non_blocking=True)
+        fd.fdllm_oproj(do, w, y)
+        hy.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, dev)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc = oproj_oracle_sample(o.cpu(), w.cpu(), 12.0)
+        cpu = {"value": v, "unit": OPROJ_UNIT, "cores": oproj_threads(), "kind": "oracle",
+               "sample": desc}
+    line = {
+        "metric": OPROJ_METRIC, "value": value, "unit": OPROJ_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config, "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": R * world / (e2e_ms / 1000.0), "unit": OPROJ_UNIT,
+                "h2d_bytes_per_step": R * H * 2, "d2h_bytes_per_step": R * H * 2,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": launches, "clocks": sampler.summary() if sampler else None,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="b32_divergent",
-                    choices=sorted(W.WORKLOADS) + sorted(W.VERIFY_WORKLOADS))
+                    choices=sorted(W.WORKLOADS) + sorted(W.VERIFY_WORKLOADS) +
+                    sorted(W.OPROJ_WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
@@ -727,6 +886,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.workload in W.VERIFY_WORKLOADS:
         return run_verify(args)
+    if args.workload in W.OPROJ_WORKLOADS:
+        return run_oproj(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_native(args)

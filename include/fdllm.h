@@ -110,7 +110,10 @@ typedef struct fdllm_cache fdllm_cache; /* opaque */
  *     slot = position.
  *   validate: 1 = copy the device metadata to the host and check it before
  *     launching (slow; for tests). Duplicate slots within a sequence and
- *     view rows writing inside [0, L_b) are only detected this way. */
+ *     view rows writing inside [0, L_b) are only detected this way.
+ *   out_bf16: 0 = `out` is fp32; 1 = `out` is bf16, each value rounded to
+ *     nearest even from the kernel's fp32 result (bf16 caches only; the
+ *     input of fdllm_oproj). */
 typedef struct {
   int32_t batch;
   int32_t total_rows;
@@ -119,6 +122,7 @@ typedef struct {
   const int32_t* seq_lens;
   const int32_t* slots;
   int32_t validate;
+  int32_t out_bf16;
 } fdllm_step;
 
 /* Creates a handle over caller-owned pools.
@@ -149,8 +153,8 @@ FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
  *     rows of its own view write in this step at positions <= its own; the
  *     two views never see each other's fresh slots. View rows must write
  *     slots >= L_b.
- *   out: DEVICE fp32 [total_rows][hidden], softmax(q k^T / sqrt(head_dim)) v
- *     per head, heads concatenated.
+ *   out: DEVICE [total_rows][hidden], fp32 (or bf16 with step->out_bf16),
+ *     softmax(q k^T / sqrt(head_dim)) v per head, heads concatenated.
  *   attn_mass: DEVICE fp32 [batch][max_blocks_per_seq * page_size] or NULL.
  *     attn_mass[b][s] = (1 / (R_b * n_heads)) * sum over heads and over the
  *     rows of b of the attention probability on slot s; zero for slots
@@ -161,7 +165,7 @@ FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
  * slot another sequence writes. */
 FDLLM_API fdllm_status fdllm_layer_step(fdllm_cache* cache, int32_t layer, const fdllm_step* step,
                               const void* x, const void* wqkv, const int32_t* positions,
-                              const int32_t* block_table, const int8_t* view_mask, float* out,
+                              const int32_t* block_table, const int8_t* view_mask, void* out,
                               float* attn_mass, void* stream);
 
 /* Next step's tracked set ([FD] paragraph 2: a fixed budget of the most
@@ -216,7 +220,7 @@ FDLLM_API fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, v
                                       int32_t layer, const fdllm_step* step, const void* x,
                                       const void* wqkv, const int32_t* positions,
                                       const int32_t* block_table, const int8_t* view_mask,
-                                      float* out, float* attn_mass, void* stream);
+                                      void* out, float* attn_mass, void* stream);
 
 /* Flash-Verify acceptance ([FD] paragraph 3: a block position is accepted
  * only when the draft view and the mask view agree and the mask view's
@@ -268,6 +272,26 @@ FDLLM_API fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_
                                       int32_t n_heads, int32_t n_bins, int32_t* bin_start,
                                       int32_t* tiles);
 
+/* Output projection of the attention block: y = attn_out W_o, bf16 in and
+ * out, fp32 accumulation (one tcgen05 GEMM launch).
+ * [FD] paragraph 1 covers a layer up to the attention output; the
+ * projection after it is the plain linear map over the heads' outputs side
+ * by side, read with the conventions of wqkv (y = x W, row-major, no bias).
+ *   attn_out: DEVICE bf16 [rows][hidden], e.g. fdllm_layer_step's out with
+ *     step->out_bf16 = 1.
+ *   w_o: DEVICE bf16 [hidden][hidden], row-major.
+ *   y: DEVICE bf16 [rows][hidden] out, each value rounded to nearest even
+ *     from the fp32 sum; must not overlap the inputs.
+ *   rows >= 0 (0 enqueues nothing); hidden a positive multiple of 256.
+ *   All three pointers 16-byte aligned.
+ *   status: DEVICE int32 or NULL; a bounded in-kernel wait that gives up
+ *     writes FDLLM_ERR_TIMEOUT there (and y is then incomplete); nothing
+ *     else writes it.
+ * Host-detectable errors return FDLLM_ERR_INVALID_ARG or
+ * FDLLM_ERR_UNSUPPORTED and enqueue nothing. */
+FDLLM_API fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t rows,
+                                   int32_t hidden, int32_t* status, void* stream);
+
 /* Synchronises `stream`, reads and clears the handle's device error word.
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
  * FDLLM_ERR_CUDA. */
@@ -280,8 +304,8 @@ FDLLM_API const char* fdllm_status_string(fdllm_status status);
 FDLLM_API const char* fdllm_last_error(void);
 
 /* Number of kernel launches the last successful fdllm_layer_step,
- * fdllm_layer_step_noalloc, fdllm_select_tracked or fdllm_verify_accept call
- * on this thread enqueued. */
+ * fdllm_layer_step_noalloc, fdllm_select_tracked, fdllm_verify_accept or
+ * fdllm_oproj call on this thread enqueued. */
 FDLLM_API int32_t fdllm_last_launch_count(void);
 
 #ifdef __cplusplus

@@ -25,7 +25,7 @@ from ._lib import (FDLLM_BF16, FDLLM_F32, FDLLM_OK, CacheConfig, FdllmError, Ste
 
 __all__ = [
     "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_layer_step_noalloc",
-    "fdllm_select_tracked", "fdllm_verify_accept", "fdllm_plan_tile_schedule",
+    "fdllm_select_tracked", "fdllm_verify_accept", "fdllm_plan_tile_schedule", "fdllm_oproj",
     "fdllm_check", "fdllm_last_launch_count", "FlashCache", "FdllmError", "load",
 ]
 
@@ -48,6 +48,15 @@ def _dev_ptr(t: Optional[torch.Tensor], dtype=None, name="tensor") -> Optional[i
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     return t.data_ptr()
+
+
+def _out_bf16(out: Optional[torch.Tensor]) -> int:
+    """1 for a bf16 `out`, 0 for fp32; anything else is refused."""
+    if out is None or out.dtype == torch.float32:
+        return 0
+    if out.dtype == torch.bfloat16:
+        return 1
+    raise ValueError(f"out must be float32 or bfloat16, got {out.dtype}")
 
 
 def _host_i32(a) -> np.ndarray:
@@ -95,11 +104,11 @@ def fdllm_layer_step(handle: int, layer: int, cu_rows: Sequence[int], seq_lens: 
     st = Step(len(sl), int(cu[-1]), int(max_blocks_per_seq),
               cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
               sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-              _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0)
+              _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0, _out_bf16(out))
     check_status(lib.fdllm_layer_step(
         handle, int(layer), ctypes.byref(st), _dev_ptr(x, None, "x"), _dev_ptr(wqkv, None, "wqkv"),
         _dev_ptr(positions, torch.int32, "positions"), _dev_ptr(block_table, torch.int32, "block_table"),
-        _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, torch.float32, "out"),
+        _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, None, "out"),
         _dev_ptr(attn_mass, torch.float32, "attn_mass"), _stream_ptr(stream)))
 
 
@@ -134,13 +143,13 @@ def fdllm_layer_step_noalloc(n_layers: int, n_heads: int, head_dim: int, page_si
     st = Step(len(sl), int(cu[-1]), int(max_blocks_per_seq),
               cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
               sl.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-              _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0)
+              _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0, _out_bf16(out))
     check_status(lib.fdllm_layer_step_noalloc(
         ctypes.byref(cfg), _dev_ptr(k_pool, tdt, "k_pool"), _dev_ptr(v_pool, tdt, "v_pool"),
         _dev_ptr(rope_cos, torch.float32, "rope_cos"), _dev_ptr(rope_sin, torch.float32, "rope_sin"),
         int(layer), ctypes.byref(st), _dev_ptr(x, None, "x"), _dev_ptr(wqkv, None, "wqkv"),
         _dev_ptr(positions, torch.int32, "positions"), _dev_ptr(block_table, torch.int32, "block_table"),
-        _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, torch.float32, "out"),
+        _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, None, "out"),
         _dev_ptr(attn_mass, torch.float32, "attn_mass"), _stream_ptr(stream)))
 
 
@@ -202,6 +211,23 @@ def fdllm_plan_tile_schedule(group_cost: Sequence[float], n_heads: int, n_bins: 
         cost.ctypes.data if n_groups else None, n_groups, int(n_heads), int(n_bins),
         bin_start.ctypes.data, tiles.ctypes.data if tiles.size else None))
     return bin_start, tiles
+
+
+def fdllm_oproj(attn_out: torch.Tensor, w_o: torch.Tensor, y: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Output projection y = attn_out W_o (see include/fdllm.h): bf16
+    [rows, hidden] times bf16 [hidden, hidden], bf16 result."""
+    lib = load()
+    rows, hidden = attn_out.shape
+    if tuple(w_o.shape) != (hidden, hidden):
+        raise ValueError(f"w_o must be [{hidden}, {hidden}], got {tuple(w_o.shape)}")
+    if y is None:
+        y = torch.empty(rows, hidden, dtype=torch.bfloat16, device=attn_out.device)
+    check_status(lib.fdllm_oproj(
+        _dev_ptr(attn_out, torch.bfloat16, "attn_out"), _dev_ptr(w_o, torch.bfloat16, "w_o"),
+        _dev_ptr(y, torch.bfloat16, "y"), int(rows), int(hidden),
+        _dev_ptr(status, torch.int32, "status"), _stream_ptr(stream)))
+    return y
 
 
 def fdllm_check(handle: int, stream=None) -> None:

@@ -37,6 +37,7 @@ class Step(ctypes.Structure):
     _fields_ = [
         ("batch", _i32), ("total_rows", _i32), ("max_blocks_per_seq", _i32),
         ("cu_rows", _i32p), ("seq_lens", _i32p), ("slots", _vp), ("validate", _i32),
+        ("out_bf16", _i32),
     ]
 
 
@@ -51,6 +52,7 @@ SIGNATURES = {
     "fdllm_verify_accept": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _vp, ctypes.c_float, _vp,
                                    _vp, _vp, _vp]),
     "fdllm_plan_tile_schedule": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "fdllm_oproj": (_i32, [_vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "fdllm_check": (_i32, [_vp, _vp]),
     "fdllm_status_string": (ctypes.c_char_p, [_i32]),
     "fdllm_last_error": (ctypes.c_char_p, []),

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfdllm.so")
-SOURCES = ["api.cu", "step_bf16.cu", "step_f32.cu", "mass_select.cu", "verify.cu"]
+SOURCES = ["api.cu", "step_bf16.cu", "step_f32.cu", "mass_select.cu", "verify.cu", "oproj.cu"]
 HEADERS = ["fdllm_internal.h", "ptx.cuh"]
 
 NVCC_FLAGS = [

@@ -91,6 +91,23 @@ bool encode_wqkv_5d(CUtensorMap* map, const void* base, uint64_t hidden, uint64_
   return r == CUDA_SUCCESS;
 }
 
+// A row-major bf16 [hidden][hidden] matrix viewed in 3 dimensions (column
+// within a 64-column block, row, column block): element (c, k, j) is
+// W[k][64 j + c]. One box {64, 64, 4} is 64 rows of 256 columns, written to
+// shared memory as four 8 KB [64 rows][128 B] sub-boxes (128-byte swizzle).
+bool encode_w_3d(CUtensorMap* map, const void* base, uint64_t hidden) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, hidden, hidden / 64};
+  cuuint64_t strides[2] = {hidden * 2, 128};
+  cuuint32_t box[3] = {64, 64, 4};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -472,7 +489,7 @@ static fdllm_status validate_device_metadata(const fdllm_cache* h, int layer, co
 
 fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* st, const void* x,
                               const void* wqkv, const int32_t* positions,
-                              const int32_t* block_table, const int8_t* view_mask, float* out,
+                              const int32_t* block_table, const int8_t* view_mask, void* out,
                               float* attn_mass, void* stream) {
   if (!h || !st) return fail(FDLLM_ERR_INVALID_ARG, "layer_step: null handle or step");
   const fdllm_cache_config& c = h->cfg;
@@ -522,6 +539,10 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   }
   if (reinterpret_cast<uintptr_t>(out) & 15)
     return fail(FDLLM_ERR_INVALID_ARG, "layer_step: out must be 16-byte aligned");
+  if (st->out_bf16 != 0 && st->out_bf16 != 1)
+    return fail(FDLLM_ERR_INVALID_ARG, "layer_step: out_bf16 must be 0 or 1");
+  if (st->out_bf16 && c.dtype != FDLLM_BF16)
+    return fail(FDLLM_ERR_UNSUPPORTED, "layer_step: bf16 out needs a bf16 cache");
 
   if (st->validate) {
     fdllm_status vs = validate_device_metadata(h, layer, st, positions, block_table, view_mask, s);
@@ -645,6 +666,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   a.page_size = c.page_size;
   a.num_pages = c.num_pages;
   a.max_position = c.max_position;
+  a.out_bf16 = st->out_bf16;
 
   int launches = 0;
   cudaError_t e = cudaSuccess;
@@ -745,6 +767,31 @@ fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_t n_groups
   return FDLLM_OK;
 }
 
+fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t rows,
+                         int32_t hidden, int32_t* status, void* stream) {
+  if (rows < 0 || hidden <= 0)
+    return fail(FDLLM_ERR_INVALID_ARG, "oproj: rows >= 0 and hidden > 0 required");
+  if (hidden % 256)
+    return fail(FDLLM_ERR_UNSUPPORTED, "oproj: hidden %d not a multiple of 256", hidden);
+  if (rows == 0) {
+    g_last_launches = 0;
+    return FDLLM_OK;
+  }
+  if (!attn_out || !w_o || !y) return fail(FDLLM_ERR_INVALID_ARG, "oproj: null pointer");
+  if ((reinterpret_cast<uintptr_t>(attn_out) | reinterpret_cast<uintptr_t>(w_o) |
+       reinterpret_cast<uintptr_t>(y)) & 15)
+    return fail(FDLLM_ERR_INVALID_ARG, "oproj: pointers must be 16-byte aligned");
+  CUtensorMap to, tw;
+  if (!encode_bf16_2d(&to, attn_out, (uint64_t)rows, (uint64_t)hidden, 128u) ||
+      !encode_w_3d(&tw, w_o, (uint64_t)hidden))
+    return fail(FDLLM_ERR_CUDA, "oproj: cuTensorMapEncodeTiled failed");
+  cudaError_t e = launch_oproj(&to, &tw, y, rows, hidden, status,
+                               reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "oproj: launch");
+  g_last_launches = 1;
+  return FDLLM_OK;
+}
+
 fdllm_status fdllm_check(fdllm_cache* h, void* stream) {
   if (!h) return fail(FDLLM_ERR_INVALID_ARG, "check: null handle");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -834,7 +881,7 @@ fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_poo
                                       const float* rope_cos, const float* rope_sin, int32_t layer,
                                       const fdllm_step* st, const void* x, const void* wqkv,
                                       const int32_t* positions, const int32_t* block_table,
-                                      const int8_t* view_mask, float* out, float* attn_mass,
+                                      const int8_t* view_mask, void* out, float* attn_mass,
                                       void* stream) {
   if (!cfg || !st) return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: null cfg or step");
   if (!k_pool || !v_pool || !rope_cos || !rope_sin)

@@ -60,7 +60,7 @@ struct StepArgs {
   const int32_t* slots;          // may be null: slot = position
   const int32_t* block_table;
   const int8_t* view;            // may be null: all plain
-  float* out;
+  void* out;                     // fp32, or bf16 when out_bf16
   float* mass_part;              // [n_heads][batch][row_stride] or null
   void* k_pool;
   void* v_pool;
@@ -73,9 +73,15 @@ struct StepArgs {
   int page_size;
   int num_pages;
   int max_position;
+  int out_bf16;
 };
 
 // Launchers (return cudaGetLastError()).
+// y = o W_o: tmap_o over o [rows][hidden] with 128-row boxes, tmap_w the
+// 3-D view of W_o {64 columns, hidden K rows, hidden / 64 column blocks}.
+cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
+                         int32_t* status, cudaStream_t stream);
+size_t oproj_smem_bytes();
 // tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
 cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
                              const void* const* tmap_x, const void* tmap_w, const void* tmap_k,

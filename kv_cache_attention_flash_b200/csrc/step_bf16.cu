@@ -1040,7 +1040,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int rr = 16 * k + j;
-          if (rr < n) a.out[(size_t)(gr0 + rr) * H + h * D + t] = any_page ? v[j] : 0.f;
+          if (rr < n) {
+            const size_t oi = (size_t)(gr0 + rr) * H + h * D + t;
+            const float ov = any_page ? v[j] : 0.f;
+            if (a.out_bf16)
+              static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(ov);
+            else
+              static_cast<float*>(a.out)[oi] = ov;
+          }
         }
       }
       ptx::tc_fence_before();

@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(NT)
       }
     }
     if (rv)
-      for (int u = 0; u < D / 32; ++u) a.out[(size_t)(r0 + r) * H + h * D + u * 32 + lane] = o[u];
+      for (int u = 0; u < D / 32; ++u)
+        static_cast<float*>(a.out)[(size_t)(r0 + r) * H + h * D + u * 32 + lane] = o[u];
   }
 }
 

@@ -414,3 +414,28 @@ def make_verify(spec: VerifySpec, seed: int, device="cpu"):
     dt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
     cu = (np.arange(B + 1) * n).astype(np.int32)
     return logits.to(dt), cu, draft.astype(np.int32)
+
+
+# ------------------------------------------------------------------ output projection
+@dataclasses.dataclass(frozen=True)
+class OprojSpec:
+    """Attention output rows of one layer step and the layer's W_o."""
+    name: str
+    rows: int
+    hidden: int
+
+
+OPROJ_WORKLOADS: Dict[str, OprojSpec] = {
+    # the batch-32 layer step's 1536 query rows at LLaDA-8B width
+    "oproj_b32": OprojSpec("oproj_b32", rows=1536, hidden=4096),
+}
+
+
+def make_oproj(spec: OprojSpec, seed: int, device="cpu"):
+    """(o [rows, hidden] bf16 ~ N(0, 1), W_o [hidden, hidden] bf16 ~
+    N(0, 0.02^2)), drawn by a seeded torch generator as float32 and cast
+    (round to nearest even)."""
+    g = _gen(seed * 1000003 + 91, device)
+    o = torch.randn(spec.rows, spec.hidden, generator=g, device=device, dtype=torch.float32)
+    w = torch.randn(spec.hidden, spec.hidden, generator=g, device=device, dtype=torch.float32) * 0.02
+    return o.to(torch.bfloat16), w.to(torch.bfloat16)
