@@ -77,10 +77,11 @@ struct StepArgs {
 };
 
 // Launchers (return cudaGetLastError()).
-// y = o W_o: tmap_o over o [rows][hidden] with 128-row boxes, tmap_w the
-// 3-D view of W_o {64 columns, hidden K rows, hidden / 64 column blocks}.
-cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
-                         int32_t* status, cudaStream_t stream);
+// y = o W_o in tiles of 128 rows x bn (256 or 128) columns: tmap_o over o
+// [rows][hidden] with 128-row boxes, tmap_w the 3-D view of W_o {64 columns,
+// hidden K rows, hidden / 64 column blocks} with boxes of bn / 64 blocks.
+cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, void* y, int rows,
+                         int hidden, int32_t* status, cudaStream_t stream);
 size_t oproj_smem_bytes();
 // tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
 cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,

@@ -8,13 +8,14 @@
 // transformer layer is a plain GEMM over the heads' outputs side by side; it
 // is read here with the conventions of Wqkv (y = x W, W row-major, no bias).
 //
-// One CTA per 128 x 256 tile of y, 192 threads:
+// One CTA per 128 x BN tile of y (BN = 256 or 128, whichever fills the SMs
+// in fewer tile-times), 192 threads:
 //   warp 0 (lane 0): TMA producer. Per 64-deep K step one box of o (128 rows
 //     x 64 columns, K-major, 128-byte swizzle) and one box of W_o (64 K rows
-//     x 4 blocks of 64 columns, N-major, 128-byte swizzle), into a 4-stage
-//     ring of 48 KB stages.
-//   warp 1 (lane 0): tcgen05.mma issuer (M128 N256 K16, A K-major, B
-//     N-major) into 256 TMEM columns; owns the TMEM allocation.
+//     x BN / 64 blocks of 64 columns, N-major, 128-byte swizzle), into a
+//     ring of 192 KB (4 stages of 48 KB, or 6 of 32 KB).
+//   warp 1 (lane 0): tcgen05.mma issuer (M128 N-BN K16, A K-major, B
+//     N-major) into BN TMEM columns; owns the TMEM allocation.
 //   warps 2-5: epilogue, one TMEM lane quadrant each: fp32 accumulator ->
 //     bf16 (round to nearest even) -> 16-byte stores of y.
 // All waits are bounded; a timeout writes FDLLM_ERR_TIMEOUT to the caller's
@@ -34,21 +35,26 @@ namespace fdllm {
 namespace {
 
 constexpr int OP_BM = 128;                                // rows of y per tile (UMMA M)
-constexpr int OP_BN = 256;                                // columns of y per tile (UMMA N)
 constexpr int OP_BK = 64;                                 // K per stage: one 128-byte span
-constexpr int OP_STAGES = 4;
 constexpr int OP_A_BYTES = OP_BM * OP_BK * 2;             // 16 KB
 constexpr int OP_BOX_BYTES = OP_BK * 64 * 2;              // 8 KB: 64 K rows x 64 columns
-constexpr int OP_B_BYTES = (OP_BN / 64) * OP_BOX_BYTES;   // 32 KB
-constexpr int OP_STAGE_BYTES = OP_A_BYTES + OP_B_BYTES;   // 48 KB
-constexpr int OP_PIPE_BYTES = OP_STAGES * OP_STAGE_BYTES;
+constexpr int OP_PIPE_BYTES = 192 * 1024;
 constexpr int OP_THREADS = 192;
-constexpr uint32_t OP_TMEM_COLS = OP_BN;
+constexpr int OP_MAX_STAGES = 6;
 constexpr uint64_t OP_WAIT_NS = 1000000000ull;            // 1 s
 
+// Per tile width BN (UMMA N): stage size and ring depth.
+template <int BN>
+struct OpCfg {
+  static constexpr int B_BYTES = (BN / 64) * OP_BOX_BYTES;
+  static constexpr int STAGE_BYTES = OP_A_BYTES + B_BYTES;      // 48 KB or 32 KB
+  static constexpr int STAGES = OP_PIPE_BYTES / STAGE_BYTES;    // 4 or 6
+  static_assert(STAGES <= OP_MAX_STAGES && STAGES * STAGE_BYTES == OP_PIPE_BYTES, "ring");
+};
+
 struct OpCtrl {
-  uint64_t full[OP_STAGES];
-  uint64_t empty[OP_STAGES];
+  uint64_t full[OP_MAX_STAGES];
+  uint64_t empty[OP_MAX_STAGES];
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -66,6 +72,7 @@ __device__ __forceinline__ bool op_wait(OpCtrl* c, uint64_t* bar, uint32_t parit
   return false;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(OP_THREADS, 1)
     oproj_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_w,
                  __nv_bfloat16* y, int rows, int hidden, int32_t* status) {
@@ -77,11 +84,13 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int m0 = blockIdx.x * OP_BM;
-  const int n0 = blockIdx.y * OP_BN;
+  constexpr int STAGES = OpCfg<BN>::STAGES;
+  constexpr int STAGE_BYTES = OpCfg<BN>::STAGE_BYTES;
+  const int n0 = blockIdx.y * BN;
   const int nkb = hidden / OP_BK;
 
   if (tid == 0) {
-    for (int s = 0; s < OP_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&ctrl->full[s], 1);
       ptx::mbar_init(&ctrl->empty[s], 1);
     }
@@ -90,7 +99,7 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&ctrl->tmem_base, OP_TMEM_COLS);
+    ptx::tmem_alloc(&ctrl->tmem_base, BN);
     ptx::tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -106,35 +115,35 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
     if (lane == 0) {
       int issued = 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % OP_STAGES;
-        const uint32_t u = kb / OP_STAGES;
+        const int s = kb % STAGES;
+        const uint32_t u = kb / STAGES;
         if (u > 0 && !op_wait(ctrl, &ctrl->empty[s], (u - 1) & 1, status)) break;
-        uint8_t* st = smem + s * OP_STAGE_BYTES;
-        ptx::mbar_arrive_expect_tx(&ctrl->full[s], OP_STAGE_BYTES);
+        uint8_t* st = smem + s * STAGE_BYTES;
+        ptx::mbar_arrive_expect_tx(&ctrl->full[s], STAGE_BYTES);
         ptx::tma_load_2d(st, &tmap_o, kb * OP_BK, m0, &ctrl->full[s]);
         ptx::tma_load_3d(st + OP_A_BYTES, &tmap_w, 0, kb * OP_BK, n0 / 64, &ctrl->full[s]);
         ++issued;
       }
       // the copies this thread issued have landed before the CTA exits
       // (they have, unless a wait timed out)
-      for (int kb = issued > OP_STAGES ? issued - OP_STAGES : 0; kb < issued; ++kb)
-        ptx::mbar_wait(&ctrl->full[kb % OP_STAGES], (kb / OP_STAGES) & 1, OP_WAIT_NS);
+      for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb)
+        ptx::mbar_wait(&ctrl->full[kb % STAGES], (kb / STAGES) & 1, OP_WAIT_NS);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(OP_BM, OP_BN, false, true);
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(OP_BM, BN, false, true);
       for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % OP_STAGES;
-        const uint32_t u = kb / OP_STAGES;
+        const int s = kb % STAGES;
+        const uint32_t u = kb / STAGES;
         if (!op_wait(ctrl, &ctrl->full[s], u & 1, status)) break;
         ptx::tc_fence_after();
-        const uint32_t a_base = ptx::smem_u32(smem + s * OP_STAGE_BYTES);
+        const uint32_t a_base = ptx::smem_u32(smem + s * STAGE_BYTES);
         const uint32_t b_base = a_base + OP_A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < OP_BK / 16; ++kk) {
           // A: K-major rows of 128 bytes, 8-row atoms 1024 bytes apart.
           const uint64_t ad = ptx::smem_desc_sw128(a_base + kk * 32, 16, 1024);
-          // B: N-major; the four 64-column boxes 8 KB apart, 8-row K groups
+          // B: N-major; the 64-column boxes 8 KB apart, 8-row K groups
           // 1024 bytes apart; a K16 slice is 16 rows = 2 KB.
           const uint64_t bd = ptx::smem_desc_sw128(b_base + kk * 2048, OP_BOX_BYTES, 1024);
           ptx::umma_f16_ss(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -155,7 +164,7 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
       __nv_bfloat16* yrow = y + (size_t)row * hidden + n0;
 #pragma unroll 1
-      for (int c0 = 0; c0 < OP_BN; c0 += 32) {
+      for (int c0 = 0; c0 < BN; c0 += 32) {
         float v[32];
         ptx::tmem_ld32(taddr + c0, v);
         ptx::tmem_ld_wait();
@@ -173,28 +182,36 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) ptx::tmem_dealloc(tmem, OP_TMEM_COLS);
+  if (warp == 1) ptx::tmem_dealloc(tmem, BN);
+}
+
+template <int BN>
+cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
+                            int32_t* status, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(oproj_kernel<BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, OP_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((rows + OP_BM - 1) / OP_BM, hidden / BN);
+  oproj_kernel<BN><<<grid, OP_THREADS, OP_SMEM_BYTES, stream>>>(
+      *reinterpret_cast<const CUtensorMap*>(tmap_o), *reinterpret_cast<const CUtensorMap*>(tmap_w),
+      reinterpret_cast<__nv_bfloat16*>(y), rows, hidden, status);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t oproj_smem_bytes() { return OP_SMEM_BYTES; }
 
-cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
-                         int32_t* status, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(oproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         OP_SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, void* y, int rows,
+                         int hidden, int32_t* status, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  dim3 grid((rows + OP_BM - 1) / OP_BM, hidden / OP_BN);
-  oproj_kernel<<<grid, OP_THREADS, OP_SMEM_BYTES, stream>>>(
-      *reinterpret_cast<const CUtensorMap*>(tmap_o), *reinterpret_cast<const CUtensorMap*>(tmap_w),
-      reinterpret_cast<__nv_bfloat16*>(y), rows, hidden, status);
-  return cudaGetLastError();
+  if (bn == 256) return launch_oproj_bn<256>(tmap_o, tmap_w, y, rows, hidden, status, stream);
+  if (bn == 128) return launch_oproj_bn<128>(tmap_o, tmap_w, y, rows, hidden, status, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fdllm

@@ -57,6 +57,19 @@ def test_oproj_full_size_sampled_rows():
     _check(W.bits_np(o)[idx], W.bits_np(w), y.float().cpu().numpy()[idx])
 
 
+def test_oproj_wide_tiles_sampled_rows():
+    """128 row tiles per SM at hidden 256: one wave of 256-column tiles
+    beats two of 128-column ones, so this runs the 256-wide instance."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rows, hidden = 128 * sms, 256
+    o, w = _case(rows, hidden, 9)
+    y = fd.fdllm_oproj(o.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    idx = np.unique(np.concatenate([[0, rows - 1], np.arange(0, rows, 997), rng.integers(0, rows, 16)]))
+    _check(W.bits_np(o)[idx], W.bits_np(w), y.float().cpu().numpy()[idx])
+
+
 def test_oproj_zero_rows_enqueues_nothing():
     o = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(256, 256, dtype=torch.bfloat16, device="cuda")
