@@ -1033,20 +1033,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ----- O^T -> out (thread t = head dimension t; the halves split rows)
       wait_bar(ctrl, &ctrl->o_done, ocount & 1, a.err, 24);
       ptx::tc_fence_after();
-      for (int k = half; k < nsub; k += 2) {
-        float v[16];
-        ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
-        ptx::tmem_ld_wait();
+      if (!a.out_bf16) {
+        float* o32 = static_cast<float*>(a.out);
+        for (int k = half; k < nsub; k += 2) {
+          float v[16];
+          ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
+          ptx::tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int rr = 16 * k + j;
-          if (rr < n) {
-            const size_t oi = (size_t)(gr0 + rr) * H + h * D + t;
-            const float ov = any_page ? v[j] : 0.f;
-            if (a.out_bf16)
-              static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(ov);
-            else
-              static_cast<float*>(a.out)[oi] = ov;
+          for (int j = 0; j < 16; ++j) {
+            const int rr = 16 * k + j;
+            if (rr < n) o32[(size_t)(gr0 + rr) * H + h * D + t] = any_page ? v[j] : 0.f;
+          }
+        }
+      } else {
+        __nv_bfloat16* o16 = static_cast<__nv_bfloat16*>(a.out);
+        for (int k = half; k < nsub; k += 2) {
+          float v[16];
+          ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int rr = 16 * k + j;
+            if (rr < n)
+              o16[(size_t)(gr0 + rr) * H + h * D + t] = __float2bfloat16_rn(any_page ? v[j] : 0.f);
           }
         }
       }
