@@ -96,3 +96,25 @@ def test_verify_empty_batch_rows():
                                         0.5, pred=pred, conf=conf)
     torch.cuda.synchronize()
     assert nacc.cpu().tolist() == [0, 0]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("vocab", [50000, 50003, 126464])
+def test_verify_large_vocab_ties_far_apart(dtype, vocab):
+    """Few rows over a large vocabulary, logits on a coarse grid with three
+    equal largest logits far apart in each row (the lowest id must win
+    across the threads and warps that saw them); an odd vocabulary takes
+    the scalar path."""
+    rng = np.random.default_rng(vocab + (dtype == "f32"))
+    R = 6
+    vals = (rng.integers(-6, 7, (R, vocab)) * 0.5).astype(np.float32)
+    # equal largest logits in different slices: the lowest id must win
+    top = float(vals.max()) + 1.0
+    for r in range(R):
+        cols = np.sort(rng.choice(vocab, size=3, replace=False))
+        vals[r, cols] = top
+    logits = torch.from_numpy(vals).to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+    cu = np.array([0, 2, 6], np.int32)
+    pred, _ = O.verify_rows(W.bits_np(logits), dtype)
+    draft = np.where(rng.random(R) < 0.8, pred, (pred + 1) % vocab).astype(np.int32)
+    _check(logits, cu, draft, 0.0)
