@@ -1,7 +1,7 @@
 """Shared helpers for the GPU parity tests: run one seeded step through the
 C-ABI library and through the CPU oracle, and compare them.
 
-Tolerances. The spec bar for bf16 is max |out_gpu - out_oracle| <=
+Tolerances. The parity bar for bf16 is max |out_gpu - out_oracle| <=
 1e-2 * RMS(out_oracle) (fp32 workloads: 1e-4), indexing bit-exact.
 
   * mode "exact" (x rows one-hot times a power of two): the projection is
@@ -39,7 +39,7 @@ from oracle import oracle as O
 
 
 @dataclasses.dataclass
-class GpuRun:
+class GpuResult:
     out: np.ndarray
     mass: np.ndarray
     tracked: np.ndarray
@@ -91,7 +91,7 @@ def run_gpu(spec, meta, x, w, kp, vp, layer=0, with_mass=True, validate=True, ca
         esl = torch.from_numpy(meta.exclude_slots if len(meta.exclude_slots) else np.zeros(1, np.int32)).to(dev)
         tracked = fd.fdllm_select_tracked(mass, sl, meta.track_k, ecu, esl).cpu().numpy()
     torch.cuda.synchronize()
-    res = GpuRun(out.cpu().numpy(), mass.cpu().numpy() if with_mass else None, tracked,
+    res = GpuResult(out.cpu().numpy(), mass.cpu().numpy() if with_mass else None, tracked,
                  W.bits_np(cache.k_pool[layer]), W.bits_np(cache.v_pool[layer]))
     if own:
         cache.close()
@@ -151,7 +151,7 @@ def tol_out(spec):
     return 1e-2 if spec.shape.dtype == "bf16" else 1e-4
 
 
-def compare(spec, meta, gpu: GpuRun, orc, kp_pre_bits, vp_pre_bits, mode="plain", probs=None,
+def compare(spec, meta, gpu: GpuResult, orc, kp_pre_bits, vp_pre_bits, mode="plain", probs=None,
             qk_spread=0.0):
     """mode: "exact" (one-hot x), "dense" (needs probs and qk_spread) or
     "plain" (plain bound everywhere; fp32 workloads)."""

@@ -51,7 +51,7 @@ def test_parity_stacked32_sampled_layers():
     stream order through one handle over the full pools, as the benchmark
     runs them; three sampled layers are checked against the oracle. One-hot
     x rows make each projection exact, so the plain bound applies."""
-    from gpu_case import GpuRun
+    from gpu_case import GpuResult
     spec = W.get_spec("stacked32_b4")
     sh = spec.shape
     meta = W.make_meta(spec, 0)
@@ -81,7 +81,7 @@ def test_parity_stacked32_sampled_layers():
     esl = torch.from_numpy(ex).to(dev)
     for l in sampled:
         tracked = fd.fdllm_select_tracked(masses[l], sl, meta.track_k, ecu, esl).cpu().numpy()
-        g = GpuRun(outs[l].cpu().numpy(), masses[l].cpu().numpy(), tracked,
+        g = GpuResult(outs[l].cpu().numpy(), masses[l].cpu().numpy(), tracked,
                    W.bits_np(cache.k_pool[l]), W.bits_np(cache.v_pool[l]))
         kb, vb = pre[l]
         o = O.layer_step(sh, kb, vb, 0, W.bits_np(xs[l]), W.bits_np(ws[l]), meta.positions,
