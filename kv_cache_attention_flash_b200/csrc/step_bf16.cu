@@ -1,13 +1,18 @@
 // Flash-Cache fused layer step for bf16 on sm_100a.
 //
-// One CTA per (row group g, head h). A row group packs whole sequences into
-// at most 128 query rows, so every fresh key/value a sequence attends to is
-// produced by the CTA that attends to it, and no grid-wide ordering is
-// needed ("Flash-dLLM: I/O-Aware KV Caching and Parallel Decoding for Fast,
-// Memory-Efficient Diffusion LLMs", ai4snews summary, paragraph 1: QKV
-// projection, RoPE and the cache write fused, K/V written to the cache from
-// on-chip memory; scheduled attention aligns each query block with its own
-// KV blocks through a block table).
+// The unit of work is a tile: one (row group g, head h). A row group packs
+// whole sequences into at most 128 query rows, so every fresh key/value a
+// sequence attends to is produced by the CTA that attends to it, and no
+// grid-wide ordering is needed ("Flash-dLLM: I/O-Aware KV Caching and
+// Parallel Decoding for Fast, Memory-Efficient Diffusion LLMs", ai4snews
+// summary, paragraph 1: QKV projection, RoPE and the cache write fused, K/V
+// written to the cache from on-chip memory; scheduled attention aligns each
+// query block with its own KV blocks through a block table). The kernel
+// runs one CTA per tile, or, when the tiles outnumber the SMs, one
+// persistent CTA per SM over a host-built list of tiles (kPersist); then
+// barrier phases, schedule counters and the TMEM allocation carry over from
+// tile to tile. TMA loads carry L2 eviction hints: x rows, Wqkv slices and
+// pass-1 K chunks are read again and stay; pass-2 K and V go first.
 //
 // Phase 1 (projection): [128 rows x H] x [H x 384], the 384 columns being
 //   this head's q | k | v blocks of Wqkv. TMA streams x and Wqkv tiles
