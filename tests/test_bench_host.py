@@ -1,0 +1,36 @@
+"""Host logic of bench.py that needs no GPU: the source hash that ties a
+committed ncu traffic figure to the kernel it was captured on, and the
+lookup that drops the figure once the sources change."""
+import os
+
+import bench
+
+
+def test_code_hash_ignores_comments_and_blank_lines(tmp_path):
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    c = tmp_path / "c.cu"
+    a.write_text("int f(int x) {\n  return x + 1;\n}\n")
+    b.write_text("// a comment\nint f(int x) {  // trailing note\n\n  return x + 1;\n}\n")
+    c.write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.code_hash(str(a)) == bench.code_hash(str(b))
+    assert bench.code_hash(str(a)) != bench.code_hash(str(c))
+
+
+def test_captured_traffic_needs_matching_sources(tmp_path, monkeypatch):
+    root = tmp_path
+    csrc = root / "kv_cache_attention_flash_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (root / "profiles").mkdir()
+    for name, body in (("step_bf16.cu", "int a;\n"), ("ptx.cuh", "int b;\n"), ("api.cu", "int c;\n")):
+        (csrc / name).write_text(body)
+    hashes = " ".join(bench.code_hash(str(csrc / n)) for n in ("step_bf16.cu", "ptx.cuh", "api.cu"))
+    (root / "profiles" / "step_bf16_demo.md").write_text(
+        f"notes\n\ntraffic_bytes_per_launch: 12345\nkernel_sources_sha256: {hashes}\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.captured_traffic("demo") == 12345.0
+    (csrc / "api.cu").write_text("int c;  // same code, new comment\n")
+    assert bench.captured_traffic("demo") == 12345.0
+    (csrc / "api.cu").write_text("int c2;\n")
+    assert bench.captured_traffic("demo") is None
+    assert bench.captured_traffic("missing") is None
