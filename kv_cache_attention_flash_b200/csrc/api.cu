@@ -75,15 +75,16 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
 // Wqkv [H][3H] bf16 viewed in 5 dimensions (column c within a 64-column
 // half, K row k, half, q/k/v block, head): element (c, k, half, blk, head)
 // is Wqkv[k][blk * H + head * head_dim + half * 64 + c]. One box
-// {64, 64, 2, 3, 1} is one head's q, k and v columns for 64 K rows, written
-// to shared memory as six 8 KB [64 rows][128 B] sub-boxes (128-byte swizzle).
+// {64, 64, 2, blocks, 1} is one head's q, k and v columns (blocks = 3), or
+// one of them (blocks = 1), for 64 K rows, written to shared memory as
+// 8 KB [64 rows][128 B] sub-boxes (128-byte swizzle).
 bool encode_wqkv_5d(CUtensorMap* map, const void* base, uint64_t hidden, uint64_t n_heads,
-                    uint64_t head_dim) {
+                    uint64_t head_dim, uint32_t blocks) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[5] = {64, hidden, head_dim / 64, 3, n_heads};
   cuuint64_t strides[4] = {3 * hidden * 2, 128, hidden * 2, head_dim * 2};
-  cuuint32_t box[5] = {64, 64, (cuuint32_t)(head_dim / 64), 3, 1};
+  cuuint32_t box[5] = {64, 64, (cuuint32_t)(head_dim / 64), blocks, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -323,6 +324,8 @@ struct fdllm_cache {
   float* mass_part;
   size_t mass_part_floats;
   int* err;
+  uint32_t* split_flags;   // [kSplitMaxTiles][k, v] for three-CTA tiles (bf16 only)
+  uint32_t split_epoch;    // value the flags of the latest such launch are set to
 };
 
 extern "C" {
@@ -403,7 +406,9 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
   if ((e = cudaMalloc(&h->rope_cos, nt * sizeof(float))) != cudaSuccess ||
       (e = cudaMalloc(&h->rope_sin, nt * sizeof(float))) != cudaSuccess ||
       (e = cudaMalloc(&h->mass_part, h->mass_part_floats * sizeof(float))) != cudaSuccess ||
-      (e = cudaMalloc(&h->err, 4 * sizeof(int))) != cudaSuccess) {
+      (e = cudaMalloc(&h->err, 4 * sizeof(int))) != cudaSuccess ||
+      (c.dtype == FDLLM_BF16 &&
+       (e = cudaMalloc(&h->split_flags, 2 * kSplitMaxTiles * sizeof(uint32_t))) != cudaSuccess)) {
     fdllm_cache_destroy(h);
     return cuda_fail(e, "cache_create: cudaMalloc");
   }
@@ -412,6 +417,9 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
       (e = cudaMemcpyAsync(h->rope_sin, sn.data(), nt * sizeof(float), cudaMemcpyHostToDevice,
                            st)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->err, 0, 4 * sizeof(int), st)) != cudaSuccess ||
+      (h->split_flags &&
+       (e = cudaMemsetAsync(h->split_flags, 0, 2 * kSplitMaxTiles * sizeof(uint32_t), st)) !=
+           cudaSuccess) ||
       (e = cudaStreamSynchronize(st)) != cudaSuccess) {
     fdllm_cache_destroy(h);
     return cuda_fail(e, "cache_create: upload");
@@ -426,6 +434,7 @@ void fdllm_cache_destroy(fdllm_cache* h) {
   cudaFree(h->rope_sin);
   cudaFree(h->mass_part);
   cudaFree(h->err);
+  cudaFree(h->split_flags);
   delete h;
 }
 
@@ -668,6 +677,8 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   a.num_pages = c.num_pages;
   a.max_position = c.max_position;
   a.out_bf16 = st->out_bf16;
+  a.split_flags = nullptr;
+  a.split_epoch = 0;
 
   int launches = 0;
   cudaError_t e = cudaSuccess;
@@ -680,10 +691,27 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
           return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (x)");
         txp[i] = &tx[i];
       }
-      if (!encode_wqkv_5d(&tw, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim))
+      if (!encode_wqkv_5d(&tw, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim, 3))
         return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv)");
-      e = launch_step_bf16(plan, tile_schedule(gcost, c.n_heads), a, txp, &tw, &h->tmap_k,
-                           &h->tmap_v, s);
+      const TileSched& ts = tile_schedule(gcost, c.n_heads);
+      // Few tiles: three CTAs per tile (q + attention, k, v), so that three
+      // times as many SMs stream the weights, when all of them fit at once.
+      const int tiles = ng * c.n_heads;
+      const int sms = sm_count();
+      CUtensorMap tw1;
+      const void* tw1p = nullptr;
+      a.split_flags = nullptr;
+      a.split_epoch = 0;
+      if (ts.n_bins == 0 && h->split_flags && sms > 0 && 3 * tiles <= sms &&
+          tiles <= kSplitMaxTiles) {
+        if (!encode_wqkv_5d(&tw1, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim, 1))
+          return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv block)");
+        tw1p = &tw1;
+        if (++h->split_epoch == 0) h->split_epoch = 1;   // flags start at 0
+        a.split_flags = h->split_flags;
+        a.split_epoch = h->split_epoch;
+      }
+      e = launch_step_bf16(plan, ts, a, txp, &tw, tw1p, &h->tmap_k, &h->tmap_v, s);
     } else {
       e = launch_step_f32(plan, a, s);
     }

@@ -131,6 +131,29 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// Flag publish / wait between CTAs of one grid: a release store and an
+// acquire load at GPU scope. The wait polls with a short sleep and gives up
+// after `budget_ns`, returning false.
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool wait_flag_gpu(const uint32_t* p, uint32_t want, uint64_t budget_ns) {
+  if (ld_acquire_gpu(p) == want) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    __nanosleep(200);
+    if (ld_acquire_gpu(p) == want) return true;
+    if (globaltimer() - t0 > budget_ns) return false;
+  }
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -261,7 +261,14 @@ struct NoSched {
 
 // kPersist: a persistent CTA runs the tiles of its schedule bin; otherwise
 // CTA i runs tile i.
-template <bool kPersist>
+// kSplit (few tiles): three CTAs per tile. CTAs 2t and 2t+1 project tile
+// t's k and v blocks only and write them to the cache, then publish them
+// through a flag (release); CTA 2T + t projects q, keeps it on chip, waits
+// for both flags (acquire, bounded) and runs the attention. Each CTA then
+// streams a third of the head's Wqkv slice. The writers come first in block
+// order and never wait, so the readers' waits end even when not every CTA
+// is resident at once.
+template <bool kPersist, bool kSplit>
 __global__ void __launch_bounds__(NTHREADS, 1)
     step_bf16_kernel(const __grid_constant__ StepPlan plan,
                      const __grid_constant__ std::conditional_t<kPersist, TileSched, NoSched> sched,
@@ -271,6 +278,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      const __grid_constant__ CUtensorMap tmap_x64,
                      const __grid_constant__ CUtensorMap tmap_x128,
                      const __grid_constant__ CUtensorMap tmap_w,
+                     const __grid_constant__ CUtensorMap tmap_w1,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
   extern __shared__ uint8_t smem_raw[];
@@ -327,6 +335,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // Tiles of this CTA (a persistent CTA runs several, one after another;
   // barrier phases, schedule counters and TMEM carry over between them).
   int t_beg = 0, t_end = 1;
+  // role: 0 = q and attention (everything when not split), 1 = k, 2 = v
+  int role = 0;
+  int tile_id = (int)blockIdx.x;
+  if constexpr (kSplit) {
+    const int T = (int)gridDim.x / 3;
+    if ((int)blockIdx.x < 2 * T) {
+      role = 1 + ((int)blockIdx.x & 1);
+      tile_id = (int)blockIdx.x >> 1;
+    } else {
+      tile_id = (int)blockIdx.x - 2 * T;
+    }
+  }
   if constexpr (kPersist) {
     t_beg = sched.bin0[blockIdx.x];
     t_end = sched.bin0[blockIdx.x + 1];
@@ -342,8 +362,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     g = sched.tile[ti] >> 8;
     h = sched.tile[ti] & 255;
   } else {   // group-major numbering (groups in order of decreasing work)
-    g = blockIdx.x / a.n_heads;
-    h = blockIdx.x % a.n_heads;
+    g = tile_id / a.n_heads;
+    h = tile_id % a.n_heads;
   }
   // sequences of this group: plan.seq_order[seq_a .. seq_b); sequence b
   // owns q rows [seq_qoff[b], seq_qoff[b] + n_b) of the 128-row tile, which
@@ -383,7 +403,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t u = kg / STAGES;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
         uint8_t* st = smem + s * STAGE_BYTES;
-        ptx::mbar_arrive_expect_tx(&ctrl->full[s], B_BYTES + x_rows * BK * 2);
+        ptx::mbar_arrive_expect_tx(&ctrl->full[s], (kSplit ? B_BYTES / 3 : B_BYTES) + x_rows * BK * 2);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (i < nbox) {
@@ -396,8 +416,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // this head's q, k and v column blocks of Wqkv, two 64-column halves
         // each: one 48 KB box of the 5-D view (column, K row, half, block,
         // head), laid out as six [64 K rows][64 columns] sub-boxes
-        ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
-                              pol_keep);
+        if constexpr (kSplit)   // this CTA's block only (q, k or v): two sub-boxes
+          ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w1, 0, kb * BK, 0, role, h, &ctrl->full[s],
+                                pol_keep);
+        else
+          ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
+                                pol_keep);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -420,11 +444,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // K groups 1024 bytes apart; K16 slice = 16 rows = 2 KB. q and k
           // (four boxes, 256 columns) go in one N=256 product, which reads
           // the A tile from shared memory once for both; v is N=128.
-          const uint64_t bqk = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
-          ptx::umma_f16_ss(tmem, ad, bqk, idesc256, (kb | kk) != 0 ? 1u : 0u);
-          const uint64_t bv = ptx::smem_desc_sw128(b_base + 4 * BOX_BYTES + kk * 2048,
-                                                   BOX_BYTES, 1024);
-          ptx::umma_f16_ss(tmem + 256, ad, bv, idesc, (kb | kk) != 0 ? 1u : 0u);
+          if constexpr (kSplit) {
+            // the one block, into its columns of the fused layout
+            const uint64_t b1 = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
+            ptx::umma_f16_ss(tmem + 128 * role, ad, b1, idesc, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint64_t bqk = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
+            ptx::umma_f16_ss(tmem, ad, bqk, idesc256, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bv = ptx::smem_desc_sw128(b_base + 4 * BOX_BYTES + kk * 2048,
+                                                     BOX_BYTES, 1024);
+            ptx::umma_f16_ss(tmem + 256, ad, bv, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
         }
         ptx::umma_commit(&ctrl->empty[s]);
       }
@@ -575,7 +605,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ctrl->sq_any[mt] = any;
     }
     // mass partials: zero (the softmax warps accumulate into them)
-    if (a.mass_part) {
+    if (a.mass_part && role == 0) {
       for (int q = 0; q < nseq; ++q) {
         float4* part = reinterpret_cast<float4*>(
             a.mass_part + ((size_t)h * plan.batch + ctrl->sq_b[q]) * plan.row_stride);
@@ -600,6 +630,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // pass (v needs no rotation, so the halves balance)
     if (warp >= 8) {
       // producer and MMA warps take no part in the epilogue
+    } else if (kSplit) {
+      if (role == 0 && warp < 4)
+        epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
+      else if (role == 1 && warp >= 4)
+        epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF);
+      else if (role == 2)
+        epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF,
+               warp < 4 ? 0 : 1, warp < 4 ? 1 : 2);
     } else if (warp < 4) {
       epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
       epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, 0, 1);
@@ -620,6 +658,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int r = idx >> 5;
       const int part = idx & 31;
       const int ch = part & 15;
+      if (kSplit && (role == 0 || (role == 1) != (part < 16))) continue;
       const int page = ctrl->row_page[r];
       if (page < 0) continue;
       const int slot = ctrl->row_slot[r];
@@ -634,6 +673,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // operand written by st.shared to the tensor cores.
   asm volatile("fence.proxy.async.global;" ::: "memory");
   fence_async_smem();
+  if constexpr (kSplit) {
+    // k/v writers: every thread's cache stores, then the flag (release)
+    __threadfence();
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    uint32_t* flag = a.split_flags + 2 * tile_id;
+    if (role != 0 && tid == 0) ptx::st_release_gpu(flag + (role - 1), a.split_epoch);
+    // q CTA: both flags (acquire), then the cache is read through TMA
+    if (role == 0 && tid == 0) {
+      bool ok = true;
+      for (int f = 0; f < 2 && ok; ++f)
+        ok = ptx::wait_flag_gpu(flag + f, a.split_epoch, WAIT_NS);
+      if (!ok) {
+        set_err(a.err, kDevTimeout, 30);
+        atomicExch(&ctrl->abort, 1);
+      }
+    }
+    __syncthreads();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -645,7 +705,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t pt_base = ptx::smem_u32(smem + PT_OFF);
   const uint32_t qrep_base = ptx::smem_u32(smem + QREP_OFF);
 
-  const int nseq_g = ctrl->nseq;
+  const int nseq_g = role == 0 ? ctrl->nseq : 0;   // k/v CTAs of a split tile stop here
   for (int si = 0; si < nseq_g; ++si) {
     const int b = ctrl->sq_b[si];
     const int n = ctrl->sq_n[si];
@@ -1102,23 +1162,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, TMEM_COLS);
 }
 
-template <bool kPersist, typename Sched>
+template <bool kPersist, bool kSplit, typename Sched>
 cudaError_t launch_kernel(int grid, const StepPlan& plan, const Sched& sched, const StepArgs& a,
-                          const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
-                          const void* tmap_v, cudaStream_t stream) {
+                          const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
+                          const void* tmap_k, const void* tmap_v, cudaStream_t stream) {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(step_bf16_kernel<kPersist>,
+    cudaError_t e = cudaFuncSetAttribute(step_bf16_kernel<kPersist, kSplit>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  step_bf16_kernel<kPersist><<<grid, NTHREADS, SMEM_BYTES, stream>>>(
+  step_bf16_kernel<kPersist, kSplit><<<grid, NTHREADS, SMEM_BYTES, stream>>>(
       plan, sched, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
       *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
       *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_k),
-      *reinterpret_cast<const CUtensorMap*>(tmap_v));
+      *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_w1),
+      *reinterpret_cast<const CUtensorMap*>(tmap_k), *reinterpret_cast<const CUtensorMap*>(tmap_v));
   return cudaGetLastError();
 }
 
@@ -1127,13 +1187,18 @@ cudaError_t launch_kernel(int grid, const StepPlan& plan, const Sched& sched, co
 size_t step_bf16_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
-                             const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
-                             const void* tmap_v, cudaStream_t stream) {
+                             const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
+                             const void* tmap_k, const void* tmap_v, cudaStream_t stream) {
   if (sched.n_bins > 0)
-    return launch_kernel<true>(sched.n_bins, plan, sched, a, tmap_x, tmap_w, tmap_k, tmap_v, stream);
+    return launch_kernel<true, false>(sched.n_bins, plan, sched, a, tmap_x, tmap_w, tmap_w,
+                                      tmap_k, tmap_v, stream);
   const int grid = plan.n_groups * a.n_heads;
   if (grid == 0) return cudaSuccess;
-  return launch_kernel<false>(grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_k, tmap_v, stream);
+  if (a.split_flags && tmap_w1)
+    return launch_kernel<false, true>(3 * grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_w1,
+                                      tmap_k, tmap_v, stream);
+  return launch_kernel<false, false>(grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_w, tmap_k,
+                                     tmap_v, stream);
 }
 
 }  // namespace fdllm
