@@ -60,6 +60,11 @@ constexpr int BOX_BYTES = BK * 64 * 2;         // 8 KB: 64 K-rows x 64 columns
 constexpr int B_BYTES = 6 * BOX_BYTES;         // q, k, v blocks, two boxes each
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES; // 64 KB
 constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
+// A split tile's CTA loads one of the q, k, v blocks (a third of B): its
+// 32 KB stages make a ring twice as deep in the same bytes.
+constexpr int SPLIT_STAGE_BYTES = A_BYTES + B_BYTES / 3;
+constexpr int SPLIT_STAGES = PIPE_BYTES / SPLIT_STAGE_BYTES;   // 6
+static_assert(SPLIT_STAGES * SPLIT_STAGE_BYTES == PIPE_BYTES, "split ring");
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 320;        // warps 0-7: epilogue / softmax (two per TMEM quadrant),
                                       // warp 8: TMA producer, warp 9: MMA issuer and TMEM owner
@@ -91,8 +96,8 @@ constexpr int QREP_OFF = PT_OFF + 32768;
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
 
 struct Ctrl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[SPLIT_STAGES];    // STAGES used, or SPLIT_STAGES in a split tile
+  uint64_t empty[SPLIT_STAGES];
   uint64_t mma_done;
   uint64_t afull[NSLOT];
   uint64_t aempty[NSLOT];
@@ -291,10 +296,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int lane = tid & 31;
   const int H = a.hidden;
   const int nkb = H / BK;
+  constexpr int kStages = kSplit ? SPLIT_STAGES : STAGES;
+  constexpr int kStageBytes = kSplit ? SPLIT_STAGE_BYTES : STAGE_BYTES;
   const int layer = plan.layer;
 
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < (kSplit ? SPLIT_STAGES : STAGES); ++s) {
       ptx::mbar_init(&ctrl->full[s], 1);
       ptx::mbar_init(&ctrl->empty[s], 1);
     }
@@ -399,10 +406,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint64_t pol_keep = ptx::policy_evict_last();
       for (int kb = 0; kb < nkb; ++kb) {
         const uint32_t kg = kstep0 + kb;
-        const int s = kg % STAGES;
-        const uint32_t u = kg / STAGES;
+        const int s = kg % kStages;
+        const uint32_t u = kg / kStages;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
-        uint8_t* st = smem + s * STAGE_BYTES;
+        uint8_t* st = smem + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&ctrl->full[s], (kSplit ? B_BYTES / 3 : B_BYTES) + x_rows * BK * 2);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -430,11 +437,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idesc256 = ptx::idesc_bf16_f32(BM, 256, false, true);
       for (int kb = 0; kb < nkb; ++kb) {
         const uint32_t kg = kstep0 + kb;
-        const int s = kg % STAGES;
-        const uint32_t u = kg / STAGES;
+        const int s = kg % kStages;
+        const uint32_t u = kg / kStages;
         if (!wait_bar(ctrl, &ctrl->full[s], u & 1, a.err, 2)) break;
         ptx::tc_fence_after();
-        const uint32_t a_base = ptx::smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t a_base = ptx::smem_u32(smem + s * kStageBytes);
         const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
