@@ -162,7 +162,11 @@ FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
  *     the statistic behind the most-attended tracking set).
  * Writes: out, attn_mass, and for every row the k/v of every head into its
  * slot; no other cache byte changes. Within one step no sequence may read a
- * slot another sequence writes. */
+ * slot another sequence writes.
+ * A handle's device workspace (mass partials, error word, the flags of
+ * steps whose tiles are split over three CTAs) serves one step at a time:
+ * steps on one handle must not run concurrently (issue them on one stream,
+ * or order the streams). */
 FDLLM_API fdllm_status fdllm_layer_step(fdllm_cache* cache, int32_t layer, const fdllm_step* step,
                               const void* x, const void* wqkv, const int32_t* positions,
                               const int32_t* block_table, const int8_t* view_mask, void* out,
