@@ -166,7 +166,16 @@ FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
  * A handle's device workspace (mass partials, error word, the flags of
  * steps whose tiles are split over three CTAs) serves one step at a time:
  * steps on one handle must not run concurrently (issue them on one stream,
- * or order the streams). */
+ * or order the streams).
+ * Steps with few tiles (three CTAs per tile fit on the SMs at once, e.g. a
+ * single sequence) split each tile over three CTAs, and the attending CTA
+ * waits, bounded to one second, for flags that the two cache-writing CTAs
+ * set. If other work on the same GPU (kernels on other streams or in other
+ * processes, a green context) keeps those CTAs off the SMs for that long,
+ * the wait gives up: that tile's out and attn_mass are then wrong and the
+ * step records FDLLM_ERR_TIMEOUT in the device error word. With
+ * step->validate = 0 the call itself still returns FDLLM_OK, so callers
+ * that share the GPU must call fdllm_check to see it. */
 FDLLM_API fdllm_status fdllm_layer_step(fdllm_cache* cache, int32_t layer, const fdllm_step* step,
                               const void* x, const void* wqkv, const int32_t* positions,
                               const int32_t* block_table, const int8_t* view_mask, void* out,
@@ -300,6 +309,25 @@ FDLLM_API fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* 
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or
  * FDLLM_ERR_CUDA. */
 FDLLM_API fdllm_status fdllm_check(fdllm_cache* cache, void* stream);
+
+/* Failure injection for tests of the error path (the paper has no
+ * counterpart). Faults are made on the host; nothing here traps, faults or
+ * hangs the GPU.
+ *   FDLLM_INJECT_SPLIT_FLAG_TIMEOUT: in the next fdllm_layer_step on `cache`
+ *     that splits its tiles over three CTAs, the attending CTAs wait for a
+ *     flag value the cache-writing CTAs never store, bounded to `wait_ns`
+ *     nanoseconds (1 .. 1e9) instead of one second. When the wait runs out
+ *     the CTA records FDLLM_ERR_TIMEOUT in the device error word and skips
+ *     its attention, issuing no further load or product; that step's out
+ *     rows are left unwritten and its attention mass is zero. The next
+ *     fdllm_check returns FDLLM_ERR_TIMEOUT and clears the word; the handle
+ *     stays usable. The injection applies once, and stays pending while
+ *     steps do not split their tiles.
+ *   FDLLM_INJECT_NONE: cancels a pending injection.
+ * Returns FDLLM_ERR_INVALID_ARG for a null handle, an unknown kind or a
+ * wait outside the range. */
+typedef enum { FDLLM_INJECT_NONE = 0, FDLLM_INJECT_SPLIT_FLAG_TIMEOUT = 1 } fdllm_inject_kind;
+FDLLM_API fdllm_status fdllm_inject_fault(fdllm_cache* cache, int32_t kind, int64_t wait_ns);
 
 /* Static description of a status code. */
 FDLLM_API const char* fdllm_status_string(fdllm_status status);

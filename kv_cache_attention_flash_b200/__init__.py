@@ -26,7 +26,8 @@ from ._lib import (FDLLM_BF16, FDLLM_F32, FDLLM_OK, CacheConfig, FdllmError, Ste
 __all__ = [
     "fdllm_cache_create", "fdllm_cache_destroy", "fdllm_layer_step", "fdllm_layer_step_noalloc",
     "fdllm_select_tracked", "fdllm_verify_accept", "fdllm_plan_tile_schedule", "fdllm_oproj",
-    "fdllm_check", "fdllm_last_launch_count", "FlashCache", "FdllmError", "load",
+    "fdllm_check", "fdllm_inject_fault", "fdllm_last_launch_count", "FlashCache", "FdllmError",
+    "load",
 ]
 
 
@@ -233,6 +234,13 @@ def fdllm_oproj(attn_out: torch.Tensor, w_o: torch.Tensor, y: Optional[torch.Ten
 def fdllm_check(handle: int, stream=None) -> None:
     """Synchronises the stream and raises FdllmError on a device-side error."""
     check_status(load().fdllm_check(handle, _stream_ptr(stream)))
+
+
+def fdllm_inject_fault(handle: int, kind: int, wait_ns: int = 0) -> None:
+    """Arms a host-made failure for the handle's next split-tile step (see
+    include/fdllm.h: the attending CTAs' bounded flag wait runs out after
+    wait_ns and the step records FDLLM_ERR_TIMEOUT)."""
+    check_status(load().fdllm_inject_fault(handle, int(kind), int(wait_ns)))
 
 
 def fdllm_last_launch_count() -> int:

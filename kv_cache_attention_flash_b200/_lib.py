@@ -18,6 +18,8 @@ FDLLM_ERR_DEVICE_BOUNDS = 4
 FDLLM_ERR_TIMEOUT = 5
 FDLLM_BF16 = 0
 FDLLM_F32 = 1
+FDLLM_INJECT_NONE = 0
+FDLLM_INJECT_SPLIT_FLAG_TIMEOUT = 1
 
 # Every function the header declares, with its ctypes signature.
 _i32 = ctypes.c_int32
@@ -54,6 +56,7 @@ SIGNATURES = {
     "fdllm_plan_tile_schedule": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "fdllm_oproj": (_i32, [_vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "fdllm_check": (_i32, [_vp, _vp]),
+    "fdllm_inject_fault": (_i32, [_vp, _i32, ctypes.c_int64]),
     "fdllm_status_string": (ctypes.c_char_p, [_i32]),
     "fdllm_last_error": (ctypes.c_char_p, []),
     "fdllm_last_launch_count": (_i32, []),

@@ -14,12 +14,27 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fdllm.h"
 #include "fdllm_internal.h"
 
 using namespace fdllm;
 
 namespace {
+
+// NVTX range over one API call, so that a profiler's timeline shows each
+// entry point around the kernels it launched (no cost without a profiler).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// Bound of the split tiles' cross-CTA flag wait (the other in-kernel waits
+// use the same one second).
+constexpr uint64_t kFlagWaitNs = 1000000000ull;
 
 thread_local std::string g_last_error;
 thread_local int32_t g_last_launches = 0;
@@ -326,6 +341,8 @@ struct fdllm_cache {
   int* err;
   uint32_t* split_flags;   // [kSplitMaxTiles][k, v] for three-CTA tiles (bf16 only)
   uint32_t split_epoch;    // value the flags of the latest such launch are set to
+  int32_t inject_kind;     // pending failure injection (fdllm_inject_fault), 0 = none
+  int64_t inject_wait_ns;
 };
 
 extern "C" {
@@ -348,6 +365,7 @@ int32_t fdllm_last_launch_count(void) { return g_last_launches; }
 
 fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, void* v_pool,
                                 void* stream, fdllm_cache** out) {
+  NvtxRange nvtx_range("fdllm_cache_create");
   if (!cfg || !out) return fail(FDLLM_ERR_INVALID_ARG, "cache_create: null cfg or out");
   *out = nullptr;
   if (!k_pool || !v_pool) return fail(FDLLM_ERR_INVALID_ARG, "cache_create: null pool");
@@ -501,6 +519,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
                               const void* wqkv, const int32_t* positions,
                               const int32_t* block_table, const int8_t* view_mask, void* out,
                               float* attn_mass, void* stream) {
+  NvtxRange nvtx_range("fdllm_layer_step");
   if (!h || !st) return fail(FDLLM_ERR_INVALID_ARG, "layer_step: null handle or step");
   const fdllm_cache_config& c = h->cfg;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -679,6 +698,8 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   a.out_bf16 = st->out_bf16;
   a.split_flags = nullptr;
   a.split_epoch = 0;
+  a.split_wait_epoch = 0;
+  a.flag_wait_ns = kFlagWaitNs;
 
   int launches = 0;
   cudaError_t e = cudaSuccess;
@@ -710,6 +731,13 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
         if (++h->split_epoch == 0) h->split_epoch = 1;   // flags start at 0
         a.split_flags = h->split_flags;
         a.split_epoch = h->split_epoch;
+        a.split_wait_epoch = h->split_epoch;
+        if (h->inject_kind == FDLLM_INJECT_SPLIT_FLAG_TIMEOUT) {
+          // a value no writer stores this launch: the attending CTAs' waits run out
+          a.split_wait_epoch = h->split_epoch ^ 0x80000000u;
+          a.flag_wait_ns = (uint64_t)h->inject_wait_ns;
+          h->inject_kind = 0;
+        }
       }
       e = launch_step_bf16(plan, ts, a, txp, &tw, tw1p, &h->tmap_k, &h->tmap_v, s);
     } else {
@@ -733,6 +761,7 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
 fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_t* seq_lens, int32_t batch,
                                   int32_t row_stride, int32_t k, const int32_t* exclude_cu,
                                   const int32_t* exclude_slots, int32_t* tracked, void* stream) {
+  NvtxRange nvtx_range("fdllm_select_tracked");
   if (!attn_mass || !seq_lens || !tracked)
     return fail(FDLLM_ERR_INVALID_ARG, "select_tracked: null attn_mass, seq_lens or tracked");
   if (batch <= 0) return fail(FDLLM_ERR_INVALID_ARG, "select_tracked: batch must be positive");
@@ -755,6 +784,7 @@ fdllm_status fdllm_verify_accept(const void* mask_logits, int32_t dtype, int32_t
                                  int32_t vocab, const int32_t* cu_rows, int32_t batch,
                                  const int32_t* draft_tokens, float tau, int32_t* pred,
                                  float* conf, int32_t* n_accepted, void* stream) {
+  NvtxRange nvtx_range("fdllm_verify_accept");
   if (dtype != FDLLM_BF16 && dtype != FDLLM_F32)
     return fail(FDLLM_ERR_INVALID_ARG, "verify_accept: unknown dtype %d", dtype);
   if (rows < 0 || batch <= 0 || vocab <= 0)
@@ -798,6 +828,7 @@ fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_t n_groups
 
 fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t rows,
                          int32_t hidden, int32_t* status, void* stream) {
+  NvtxRange nvtx_range("fdllm_oproj");
   if (rows < 0 || hidden <= 0)
     return fail(FDLLM_ERR_INVALID_ARG, "oproj: rows >= 0 and hidden > 0 required");
   if (hidden % 256)
@@ -831,7 +862,24 @@ fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t
   return FDLLM_OK;
 }
 
+fdllm_status fdllm_inject_fault(fdllm_cache* h, int32_t kind, int64_t wait_ns) {
+  if (!h) return fail(FDLLM_ERR_INVALID_ARG, "inject_fault: null handle");
+  if (kind == FDLLM_INJECT_NONE) {
+    h->inject_kind = 0;
+    return FDLLM_OK;
+  }
+  if (kind != FDLLM_INJECT_SPLIT_FLAG_TIMEOUT)
+    return fail(FDLLM_ERR_INVALID_ARG, "inject_fault: unknown kind %d", kind);
+  if (wait_ns < 1 || wait_ns > (int64_t)kFlagWaitNs)
+    return fail(FDLLM_ERR_INVALID_ARG, "inject_fault: wait_ns %lld outside [1, 1e9]",
+                (long long)wait_ns);
+  h->inject_kind = kind;
+  h->inject_wait_ns = wait_ns;
+  return FDLLM_OK;
+}
+
 fdllm_status fdllm_check(fdllm_cache* h, void* stream) {
+  NvtxRange nvtx_range("fdllm_check");
   if (!h) return fail(FDLLM_ERR_INVALID_ARG, "check: null handle");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(s);
@@ -922,6 +970,7 @@ fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_poo
                                       const int32_t* positions, const int32_t* block_table,
                                       const int8_t* view_mask, void* out, float* attn_mass,
                                       void* stream) {
+  NvtxRange nvtx_range("fdllm_layer_step_noalloc");
   if (!cfg || !st) return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: null cfg or step");
   if (!k_pool || !v_pool || !rope_cos || !rope_sin)
     return fail(FDLLM_ERR_INVALID_ARG, "layer_step_noalloc: null pool or RoPE table");
@@ -1003,10 +1052,17 @@ fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_poo
   if ((e = cudaMemsetAsync(h.err, 0, sizeof(w), reinterpret_cast<cudaStream_t>(stream))) !=
       cudaSuccess)
     return cuda_fail(e, "layer_step_noalloc: clear error word");
+  // The word is shared by every call on this device: what it holds may have
+  // been recorded by an earlier call made with validate = 0.
   if (w[0] == kDevTimeout)
-    return fail(FDLLM_ERR_TIMEOUT, "device: bounded wait timed out (site %d)", w[1]);
-  return fail(FDLLM_ERR_DEVICE_BOUNDS, "device: metadata out of range (code %d, detail %d)", w[0],
-              w[1]);
+    return fail(FDLLM_ERR_TIMEOUT,
+                "device: bounded wait timed out (site %d), in this call or an earlier "
+                "validate = 0 call on this device",
+                w[1]);
+  return fail(FDLLM_ERR_DEVICE_BOUNDS,
+              "device: metadata out of range (code %d, detail %d), in this call or an earlier "
+              "validate = 0 call on this device",
+              w[0], w[1]);
 }
 
 }  // extern "C"

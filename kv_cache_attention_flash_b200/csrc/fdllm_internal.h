@@ -1,6 +1,7 @@
 // Internal declarations shared by the host API and the kernels.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -79,6 +80,10 @@ struct StepArgs {
   // split_epoch when that block is in the cache; null = one CTA per tile
   uint32_t* split_flags;
   uint32_t split_epoch;
+  // value the attending CTA of a split tile waits for (split_epoch, except
+  // under failure injection) and the bound of that wait in nanoseconds
+  uint32_t split_wait_epoch;
+  uint64_t flag_wait_ns;
 };
 
 // Launchers (return cudaGetLastError()).
@@ -108,5 +113,21 @@ cudaError_t launch_verify_accept(const void* logits, bool bf16, int rows, int vo
                                  cudaStream_t stream);
 
 size_t step_bf16_smem_bytes();
+
+// Opts `fn` into `bytes` of dynamic shared memory on the current device.
+// The attribute lives in each device's context, so the record of which
+// devices are done is per device (a bit per device id below 64; others set
+// it on every launch). Setting it twice is harmless, so concurrent first
+// calls need no lock.
+inline cudaError_t opt_in_smem(const void* fn, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t{1} << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 }  // namespace fdllm

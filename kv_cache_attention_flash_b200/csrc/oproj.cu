@@ -188,13 +188,10 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
 template <int BN>
 cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
                             int32_t* status, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(oproj_kernel<BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, OP_SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = opt_in_smem(reinterpret_cast<const void*>(oproj_kernel<BN>), OP_SMEM_BYTES,
+                              attr_done);
+  if (e != cudaSuccess) return e;
   dim3 grid((rows + OP_BM - 1) / OP_BM, hidden / BN);
   oproj_kernel<BN><<<grid, OP_THREADS, OP_SMEM_BYTES, stream>>>(
       *reinterpret_cast<const CUtensorMap*>(tmap_o), *reinterpret_cast<const CUtensorMap*>(tmap_w),

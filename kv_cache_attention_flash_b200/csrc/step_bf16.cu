@@ -692,7 +692,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (role == 0 && tid == 0) {
       bool ok = true;
       for (int f = 0; f < 2 && ok; ++f)
-        ok = ptx::wait_flag_gpu(flag + f, a.split_epoch, WAIT_NS);
+        ok = ptx::wait_flag_gpu(flag + f, a.split_wait_epoch, a.flag_wait_ns);
       if (!ok) {
         set_err(a.err, kDevTimeout, 30);
         atomicExch(&ctrl->abort, 1);
@@ -712,7 +712,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t pt_base = ptx::smem_u32(smem + PT_OFF);
   const uint32_t qrep_base = ptx::smem_u32(smem + QREP_OFF);
 
-  const int nseq_g = role == 0 ? ctrl->nseq : 0;   // k/v CTAs of a split tile stop here
+  // k/v CTAs of a split tile stop here, and so does an attending CTA whose
+  // wait for them gave up: it issues no load and no product, so nothing is
+  // left in flight (its out rows stay unwritten, its mass partials zero, and
+  // the error word holds the timeout)
+  const bool gave_up = kSplit && *reinterpret_cast<volatile int*>(&ctrl->abort) != 0;
+  const int nseq_g = (role == 0 && !gave_up) ? ctrl->nseq : 0;
   for (int si = 0; si < nseq_g; ++si) {
     const int b = ctrl->sq_b[si];
     const int n = ctrl->sq_n[si];
@@ -1173,13 +1178,10 @@ template <bool kPersist, bool kSplit, typename Sched>
 cudaError_t launch_kernel(int grid, const StepPlan& plan, const Sched& sched, const StepArgs& a,
                           const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
                           const void* tmap_k, const void* tmap_v, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(step_bf16_kernel<kPersist, kSplit>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = opt_in_smem(reinterpret_cast<const void*>(step_bf16_kernel<kPersist, kSplit>),
+                              SMEM_BYTES, attr_done);
+  if (e != cudaSuccess) return e;
   step_bf16_kernel<kPersist, kSplit><<<grid, NTHREADS, SMEM_BYTES, stream>>>(
       plan, sched, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
       *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),

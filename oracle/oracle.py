@@ -226,8 +226,15 @@ def layer_step_from_projection(shape, k_pool, v_pool, layer, a, positions, slots
             if probs is not None:
                 probs[(b, h)] = (keys, P)
             # 6. attention mass: mean over heads and rows  [FD ¶2]
-            np.add.at(mass[b], keys, P.sum(axis=0) / ((r1 - r0) * nh))
+            np.add.at(mass[b], keys, P.sum(axis=0) * mass_weight(r1 - r0, nh))
     return out, mass, k_pool, v_pool
+
+
+def mass_weight(n_rows: int, n_heads: int) -> float:
+    """Weight of one probability in the attention mass: the mass is the
+    mean over the sequence's rows and over the heads [FD ¶2], so each of the
+    n_rows * n_heads probability rows counts 1 / (n_rows * n_heads)."""
+    return 1.0 / (n_rows * n_heads)
 
 
 def softmax_rows(S: np.ndarray, vis: np.ndarray) -> np.ndarray:

@@ -1,24 +1,22 @@
 """Shared helpers for the GPU parity tests: run one seeded step through the
 C-ABI library and through the CPU oracle, and compare them.
 
-Tolerances. The parity bar for bf16 is max |out_gpu - out_oracle| <=
-1e-2 * RMS(out_oracle) (fp32 workloads: 1e-4), indexing bit-exact.
+Tolerances. The parity bar for `out` is the plain one in every mode:
+max |out_gpu - out_oracle| <= 1e-2 * RMS(out_oracle) for bf16 workloads
+(1e-4 for fp32), indexing bit-exact. Each comparison prints its measured
+max|err|/RMS.
 
   * mode "exact" (x rows one-hot times a power of two): the projection is
     exact in fp32 and fp64 alike, so no bf16 rounding decision can differ.
-    out must meet the plain bar; written v must be bit-identical; written k
-    (rotated in fp32 on the GPU, fp64 in the oracle) within 1 bf16 ulp plus
-    1e-5 * RMS for values next to zero.
-  * mode "dense" (x ~ N(0,1)): the bf16 codes of the fresh q/k/v are decided
-    from an fp32 accumulator on the GPU and an fp64 one in the oracle; where
-    the two land on opposite sides of a rounding midpoint both codes are
-    correct. Written values: 1 bf16 ulp plus 1e-3 * RMS (the size of an fp32
-    accumulation error over K = 4096, which exceeds one ulp of values near
-    zero). out, per element: 1e-2 * RMS + sum over fresh keys of P * ulp(v)
-    (the largest effect of one-ulp changes of the fresh v, from the oracle's
-    own P and v) + 2 * the spread that the same fp32-vs-fp64 choice for q and
-    k alone produces inside the oracle (projection re-accumulated in float32
-    by numpy for the q and k columns).
+    Written v must be bit-identical; written k (rotated in fp32 on the GPU,
+    fp64 in the oracle) within 1 bf16 ulp plus 1e-5 * RMS for values next
+    to zero.
+  * mode "dense" (x ~ N(0,1), the workloads' input distribution): the bf16
+    codes of the fresh q/k/v are decided from an fp32 accumulator on the GPU
+    and an fp64 one in the oracle; where the two land on opposite sides of a
+    rounding midpoint both codes are correct. Written values: 1 bf16 ulp
+    plus 1e-3 * RMS (the size of an fp32 accumulation error over K = 4096,
+    which exceeds one ulp of values near zero).
   * attn_mass: |gpu - oracle| <= 1e-3 * |oracle| + 1e-6.
   * cache: every byte outside the written slots bit-identical to the
     pre-state.
@@ -104,71 +102,31 @@ def run_oracle(spec, meta, x, w, kp, vp, probs=None):
                         meta.view, probs=probs)
 
 
-def qk_rounding_spread(spec, meta, x, w, kp, vp, o_out):
-    """max |out' - out| where out' re-accumulates the q and k columns of the
-    projection in float32 (a legitimate fp32 implementation's rounding
-    choices) and keeps everything else of the oracle."""
-    sh = spec.shape
-    H = sh.hidden
-    a = O.project(sh, W.bits_np(x), W.bits_np(w))
-    xf = O.decode(W.bits_np(x), sh.dtype).astype(np.float32)
-    wf = O.decode(W.bits_np(w), sh.dtype).astype(np.float32)
-    a[:, :2 * H] = (xf @ wf[:, :2 * H]).astype(np.float64)
-    alt = O.layer_step_from_projection(sh, W.bits_np(kp), W.bits_np(vp), 0, a, meta.positions,
-                                       meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table,
-                                       meta.view)[0]
-    return float(np.max(np.abs(alt - o_out)))
-
-
 def bf16_ulp(v):
     """Spacing of bfloat16 numbers at |v| (normal range)."""
     a = np.maximum(np.abs(v), 2.0 ** -126)
     return 2.0 ** (np.floor(np.log2(a)) - 7)
 
 
-def fresh_v_sensitivity(spec, meta, probs, o_vp):
-    """Per output element: sum over this step's fresh keys j of
-    P_rj * ulp(v_j,d), the largest change a one-ulp change of every fresh v
-    can make."""
-    sh = spec.shape
-    D, ps = sh.head_dim, sh.page_size
-    R = meta.total_rows
-    t = np.zeros((R, sh.hidden))
-    for (b, h), (keys, P) in probs.items():
-        r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
-        fresh = set(int(s) for s in meta.slots[r0:r1])
-        sel = [i for i, k in enumerate(keys) if int(k) in fresh]
-        if not sel:
-            continue
-        ks = keys[sel]
-        pages = meta.block_table[b, ks // ps]
-        v = O.decode(o_vp[0, pages, h, ks % ps, :], sh.dtype)       # [nf, D]
-        t[r0:r1, h * D:(h + 1) * D] += P[:, sel] @ bf16_ulp(v)
-    return t
-
-
 def tol_out(spec):
     return 1e-2 if spec.shape.dtype == "bf16" else 1e-4
 
 
-def compare(spec, meta, gpu: GpuResult, orc, kp_pre_bits, vp_pre_bits, mode="plain", probs=None,
-            qk_spread=0.0):
-    """mode: "exact" (one-hot x), "dense" (needs probs and qk_spread) or
-    "plain" (plain bound everywhere; fp32 workloads)."""
+def compare(spec, meta, gpu: GpuResult, orc, kp_pre_bits, vp_pre_bits, mode="plain", label=None):
+    """mode: "exact" (one-hot x), "dense" (N(0,1) x) or "plain" (fp32
+    workloads). `out` meets the plain bar in every mode. Returns
+    max|err|/RMS of `out`."""
     o_out, o_mass, o_kp, o_vp = orc
     sh = spec.shape
     # out
     rms = float(np.sqrt(np.mean(o_out ** 2)))
     diff = np.abs(gpu.out - o_out)
-    err = float(np.max(diff))
+    err = float(np.max(diff)) if diff.size else 0.0
+    ratio = err / max(rms, 1e-30)
+    print(f"[parity] {label or spec.name} mode={mode}: max|err|/RMS = {ratio:.3e} "
+          f"(bar {tol_out(spec):.0e})")
     assert np.all(np.isfinite(gpu.out)), "non-finite output"
-    if mode != "dense" or sh.dtype != "bf16":
-        assert err <= tol_out(spec) * rms, f"out: max err {err:.3e} > {tol_out(spec)} * rms {rms:.3e}"
-    else:
-        extra = fresh_v_sensitivity(spec, meta, probs, o_vp)
-        bad = diff > tol_out(spec) * rms + extra + 2.0 * qk_spread
-        assert not np.any(bad), (f"out: {int(bad.sum())} elements over the dense bound; "
-                                 f"max err/rms {err / rms:.3e}, qk spread/rms {qk_spread / rms:.3e}")
+    assert err <= tol_out(spec) * rms, f"out: max err {err:.3e} > {tol_out(spec)} * rms {rms:.3e}"
     # cache bytes
     wm = written_mask(meta, sh)
     full = np.broadcast_to(wm[:, None, :, None], gpu.k_pool.shape)
@@ -207,4 +165,4 @@ def compare(spec, meta, gpu: GpuResult, orc, kp_pre_bits, vp_pre_bits, mode="pla
             kth = min(o_mass[b, j] for j in b_set)
             for j in a_set ^ b_set:
                 assert abs(o_mass[b, j] - kth) <= 1e-3 * kth, f"seq {b}: slot {j} is not a near-tie"
-    return err / max(rms, 1e-30)
+    return ratio

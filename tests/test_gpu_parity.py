@@ -10,19 +10,15 @@ import kv_cache_attention_flash_b200 as fd
 from kv_cache_attention_flash_b200 import workloads as W
 from oracle import oracle as O
 
-from gpu_case import build_inputs, compare, qk_rounding_spread, run_gpu, run_oracle
+from gpu_case import build_inputs, compare, run_gpu, run_oracle
 
 
 def check_dense(spec, meta, x, w, kp, vp, g):
-    """Compare a dense-x GPU run with the oracle (mode "dense")."""
-    probs = {}
-    o = run_oracle(spec, meta, x, w, kp, vp, probs=probs)
-    if spec.shape.dtype == "bf16":
-        spread = qk_rounding_spread(spec, meta, x, w, kp, vp, o[0])
-        compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="dense", probs=probs,
-                qk_spread=spread)
-    else:
-        compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="plain")
+    """Compare a dense-x GPU run with the oracle: the plain 1e-2 * RMS bar
+    on out (1e-4 for fp32), cache values within one bf16 ulp."""
+    o = run_oracle(spec, meta, x, w, kp, vp)
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp),
+            mode="dense" if spec.shape.dtype == "bf16" else "plain")
 
 pytestmark = pytest.mark.gpu
 

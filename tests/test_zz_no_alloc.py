@@ -7,10 +7,10 @@ entry point serves them: it takes the pools and RoPE tables the caller owns,
 and keeps its only scratch (per-head attention-mass partials and an error
 word) in a fixed array inside the library's device image.
 
-These tests call it through the C ABI and compare it with fdllm_layer_step
-on the same inputs, twice in a row (the second call runs on the cache the
-first one wrote, and on whatever the first call left in the shared scratch),
-within the parity tests' tolerances. This file sorts last so that a run
+These tests call it through the C ABI twice in a row (the second call runs
+on the cache the first one wrote, and on whatever the first call left in the
+shared scratch). Each call is compared with fdllm_layer_step on the same
+inputs and with the CPU oracle, within the parity tests' tolerances. This file sorts last so that a run
 stopping at the first failure has run every other test before it.
 """
 import ctypes
@@ -22,6 +22,9 @@ import torch
 import kv_cache_attention_flash_b200 as fd
 from kv_cache_attention_flash_b200 import _lib
 from kv_cache_attention_flash_b200 import workloads as W
+from oracle import oracle as O
+
+from gpu_case import GpuResult, compare
 
 # Capacity of the library's fixed mass scratch, in floats (8 MiB less a
 # 256-byte header for the error word).
@@ -97,6 +100,12 @@ def test_noalloc_matches_layer_step_twice(name):
     def bits(t):
         return W.bits_np(t[0])
 
+    # the oracle's own cache state, carried from call to call
+    o_kp, o_vp = W.bits_np(kp), W.bits_np(vp)
+    sl_d = torch.from_numpy(meta.seq_lens).to(dev)
+    ecu_d = torch.from_numpy(meta.exclude_cu).to(dev)
+    esl_d = torch.from_numpy(meta.exclude_slots if len(meta.exclude_slots)
+                             else np.zeros(1, np.int32)).to(dev)
     for call, x in enumerate(xs):
         out_a, mass_a = cache.step(0, meta.cu_rows, meta.seq_lens, x, w, pos, bt, view_mask=view,
                                    slots=slots, validate=True)
@@ -112,6 +121,14 @@ def test_noalloc_matches_layer_step_twice(name):
         assert_close(spec, out_a.cpu().numpy(), mass_a.cpu().numpy(), bits(cache.k_pool),
                      bits(cache.v_pool), out_b.cpu().numpy(), mass_b.cpu().numpy(), bits(kb),
                      bits(vb), f"{name} call {call + 1}")
+        # and against the oracle directly
+        orc = O.layer_step(sh, o_kp, o_vp, 0, W.bits_np(x), W.bits_np(w), meta.positions,
+                           meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table, meta.view)
+        tracked = fd.fdllm_select_tracked(mass_b, sl_d, meta.track_k, ecu_d, esl_d).cpu().numpy()
+        g = GpuResult(out_b.cpu().numpy(), mass_b.cpu().numpy(), tracked, bits(kb), bits(vb))
+        compare(spec, meta, g, orc, o_kp, o_vp, mode="dense" if sh.dtype == "bf16" else "plain",
+                label=f"{name} no-alloc call {call + 1}")
+        o_kp, o_vp = orc[2], orc[3]
     cache.close()
 
 
