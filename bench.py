@@ -59,28 +59,22 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# DRAM traffic of the fused step kernel, per launch, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), with the code hashes of the
+# sources it was captured on: the kernel, its PTX helpers and the host code
+# that plans its launch. The figure is reported only while all three match.
+CAPTURED_TRAFFIC = {}
+
+
 def captured_traffic(name: str):
-    """DRAM bytes per launch of the step kernel from the committed ncu
-    summary for this workload, if the kernel sources are unchanged since the
-    capture (else None)."""
-    path = os.path.join(ROOT, "profiles", f"step_bf16_{name}.md")
-    if not os.path.exists(path):
-        return None
-    txt = open(path).read()
-    want = None
-    traffic = None
-    for line in txt.splitlines():
-        if line.startswith("traffic_bytes_per_launch:"):
-            traffic = float(line.split(":", 1)[1])
-        if line.startswith("kernel_sources_sha256:"):
-            want = line.split(":", 1)[1].split()
-    if traffic is None or want is None:
+    """DRAM bytes per launch of the step kernel for this workload, if a
+    capture of the current kernel sources is recorded above (else None)."""
+    rec = CAPTURED_TRAFFIC.get(name)
+    if rec is None:
         return None
     csrc = os.path.join(ROOT, "kv_cache_attention_flash_b200", "csrc")
-    # the kernel, its PTX helpers and the host code that plans its launch
-    # (row groups and the tile schedule decide what each CTA reads)
     have = [code_hash(os.path.join(csrc, f)) for f in ("step_bf16.cu", "ptx.cuh", "api.cu")]
-    return traffic if have == want else None
+    return rec["bytes"] if have == rec["sources"] else None
 
 
 def code_hash(path: str) -> str:
@@ -228,20 +222,22 @@ class Workload:
         self.tracked = torch.empty(m.batch, m.track_k, dtype=torch.int32, device=device)
         self.launches_per_step = None
 
-    def step(self, x_list=None, ev=None):
+    def step(self, x_list=None, ev=None, layer_span=False):
         """One pass of the hot path; returns the number of kernels launched.
-        If `ev` is given, events are recorded around each layer step."""
+        If `ev` is given, events are recorded around the first layer step, or
+        (layer_span) from the first layer step to the end of the last."""
         fd = self.fd
         m = self.meta
         n = 0
         xs = x_list if x_list is not None else self.x
-        for l in range(self.n_layers):
-            if ev is not None:
+        nl = self.n_layers
+        for l in range(nl):
+            if ev is not None and l == 0:
                 ev[0].record()
             fd.fdllm_layer_step(self.cache.handle, l, m.cu_rows, m.seq_lens, m.max_blocks, xs[l],
                                 self.w[l], self.pos, self.bt, self.view, self.out, self.mass,
                                 self.slots)
-            if ev is not None:
+            if ev is not None and (l == nl - 1 or not layer_span):
                 ev[1].record()
                 ev = None
             n += fd.fdllm_last_launch_count()
@@ -249,6 +245,129 @@ class Workload:
                                 self.tracked)
         n += fd.fdllm_last_launch_count()
         return n
+
+
+# ------------------------------------------------------------------ unfused baseline
+class UnfusedStep:
+    """The pages' prior art for one layer step, as separate PyTorch launches
+    whose intermediates all round-trip HBM ("Flash-dLLM: I/O-Aware KV Caching
+    and Parallel Decoding for Fast, Memory-Efficient Diffusion LLMs", ai4snews
+    summary, paragraph 1: before Flash-Cache the per-layer cache update was
+    a chain of separate kernel launches): a cuBLAS GEMM x Wqkv, RoPE as
+    elementwise ops, index_put_ of k and v into the paged pools, a gather of
+    every sequence's keys and values through the block table, then scores,
+    masked softmax and P V on a padded batch, and the attention mass from
+    the probabilities. Same inputs, pool layout and results (within the
+    parity bar) as the fused step; it exists only to measure what the fusion
+    saves. The projection and the scores take bf16 operands with fp32
+    results (cuBLAS), so q and k are rounded once, after RoPE, as in the
+    fused step; P V runs in fp32 with TF32 allowed, which is exact for the
+    bf16-valued v and rounds P to 11 bits.
+
+    The padded shapes and the row / key index tensors depend only on cu_rows
+    and seq_lens (host metadata, as in the fused path) and are built once;
+    everything that depends on the device inputs (positions, slots, views,
+    block table) is computed on the device in every step."""
+
+    def __init__(self, spec, meta, device):
+        sh = spec.shape
+        self.sh, self.meta, self.dev = sh, meta, device
+        D, ps = sh.head_dim, sh.page_size
+        half = D // 2
+        inv = np.float64(np.float32(sh.rope_theta)) ** (-2.0 * np.arange(half) / D)
+        phi = np.arange(meta.max_position, dtype=np.float64)[:, None] * inv[None, :]
+        self.cos = torch.from_numpy(np.cos(phi).astype(np.float32)).to(device)
+        self.sin = torch.from_numpy(np.sin(phi).astype(np.float32)).to(device)
+        B = meta.batch
+        cu = meta.cu_rows
+        n = np.diff(cu)
+        self.Rmax = max(1, int(n.max()))
+        kb = [max(int(meta.seq_lens[b]), int(meta.slots[cu[b]:cu[b + 1]].max()) + 1 if n[b] else 0)
+              for b in range(B)]
+        self.Kmax = max(1, max(kb))
+        rowidx = np.full((B, self.Rmax), -1, np.int64)
+        rowb = np.zeros(meta.total_rows, np.int64)
+        for b in range(B):
+            rowidx[b, :n[b]] = np.arange(cu[b], cu[b + 1])
+            rowb[cu[b]:cu[b + 1]] = b
+        kslot = np.tile(np.arange(self.Kmax, dtype=np.int64), (B, 1))
+        kvalid = kslot < np.array(kb)[:, None]
+        wgt = np.where(n > 0, 1.0 / np.maximum(n, 1) / sh.n_heads, 0.0)
+        self.rowvalid = torch.from_numpy(rowidx >= 0).to(device)
+        self.rowidx = torch.from_numpy(np.maximum(rowidx, 0)).to(device)
+        self.rowb = torch.from_numpy(rowb).to(device)
+        self.kslot = torch.from_numpy(kslot).to(device)
+        self.kvalid = torch.from_numpy(kvalid).to(device)
+        self.seq_lens = torch.from_numpy(meta.seq_lens.astype(np.int64)).to(device)
+        self.wgt = torch.from_numpy(wgt.astype(np.float32)).to(device)
+        self.scale = 1.0 / float(np.sqrt(D))
+
+    def _rope(self, u, c, s):
+        half = self.sh.head_dim // 2
+        u = u.float()
+        a, b = u[..., :half], u[..., half:]
+        return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+
+    def step(self, layer, k_pool, v_pool, x, w, pos, slots, view, bt, out, mass):
+        sh, meta = self.sh, self.meta
+        H, nh, D, ps = sh.hidden, sh.n_heads, sh.head_dim, sh.page_size
+        R, B = meta.total_rows, meta.batch
+        bf = torch.bfloat16
+        # 1. projection (cuBLAS, bf16 in, fp32 out so that q and k are rounded
+        # once, after RoPE, as in the fused step), q, k, v through HBM
+        qkv = torch.mm(x, w, out_dtype=torch.float32) if x.is_cuda else x.float() @ w.float()
+        q = qkv[:, :H].view(R, nh, D)
+        k = qkv[:, H:2 * H].view(R, nh, D)
+        v = qkv[:, 2 * H:].view(R, nh, D)
+        # 2. RoPE (elementwise launches)
+        p = pos.long()
+        c = self.cos[p][:, None, :]
+        s = self.sin[p][:, None, :]
+        qr = self._rope(q, c, s).to(bf)
+        kr = self._rope(k, c, s).to(bf)
+        # 3. cache write through the block table (index_put_)
+        sl = slots.long()
+        btl = bt.long()
+        page = btl[self.rowb, sl // ps]
+        off = sl % ps
+        kp, vp = k_pool[layer], v_pool[layer]
+        kp[page, :, off] = kr
+        vp[page, :, off] = v.to(bf)
+        # 4. gather every sequence's keys / values (padded batch)
+        ks = self.kslot
+        kpage = btl.gather(1, torch.clamp(ks // ps, max=btl.shape[1] - 1))
+        kpage = torch.where(self.kvalid, kpage, torch.zeros_like(kpage))
+        K = kp[kpage, :, ks % ps]                     # [B, Kmax, nh, D]
+        V = vp[kpage, :, ks % ps]
+        Q = qr[self.rowidx]                           # [B, Rmax, nh, D]
+        # 5. visibility: context slots, plus own-view fresh slots at earlier
+        # or equal positions
+        rv = view.long()[self.rowidx]
+        rp = p[self.rowidx]
+        wv = torch.full((B, self.Kmax), -1, dtype=torch.long, device=self.dev)
+        wp = torch.zeros((B, self.Kmax), dtype=torch.long, device=self.dev)
+        wv[self.rowb, sl] = view.long()
+        wp[self.rowb, sl] = p
+        ctx = ks < self.seq_lens[:, None]
+        own = (wv[:, None, :] == rv[:, :, None]) & (rv[:, :, None] != 0) & \
+              (wp[:, None, :] <= rp[:, :, None])
+        vis = (ctx[:, None, :] | own) & self.kvalid[:, None, :] & self.rowvalid[:, :, None]
+        # 6. scores, masked softmax, P V
+        Qb = Q.permute(0, 2, 1, 3).reshape(B * nh, self.Rmax, D)
+        Kb = K.permute(0, 2, 3, 1).reshape(B * nh, D, self.Kmax)
+        S = (torch.bmm(Qb, Kb, out_dtype=torch.float32) if Qb.is_cuda
+             else torch.bmm(Qb.float(), Kb.float()))
+        S = S.view(B, nh, self.Rmax, self.Kmax) * self.scale
+        S = S.masked_fill(~vis[:, None], float("-inf"))
+        P = torch.nan_to_num(torch.softmax(S, dim=-1), nan=0.0)
+        O = torch.matmul(P, V.permute(0, 2, 1, 3).float())    # [B, nh, Rmax, D]
+        o = O.permute(0, 2, 1, 3).reshape(B, self.Rmax, H)
+        out[self.rowidx[self.rowvalid]] = o[self.rowvalid]
+        # 7. attention mass: mean over heads and rows
+        if mass is not None:
+            m = P.sum(dim=(1, 2)) * self.wgt[:, None]
+            mass.zero_()
+            mass[:, :self.Kmax] = m
 
 
 # ------------------------------------------------------------------ CPU baseline
@@ -402,31 +521,65 @@ def e2e_measure(wl: Workload, steps: int):
 
 # ------------------------------------------------------------------ main arms
 def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores.
+    Every step is one bounded sample of the workload (the first sequences
+    of layer 0, as many as fit about 20 s / (steps + warm-up) of oracle
+    time, at least one), and every step is timed whole, so ms_per_step x
+    steps is the time the run spent in timed steps."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
+    from oracle import oracle as O
     spec = W.get_spec(args.workload)
     meta = W.make_meta(spec, args.seed)
-    budget = max(2.0, 20.0 / max(1, args.steps + args.warmup))
-    vals = []
-    desc = ""
-    threads = 1
+    xb, wb, kb, vb = oracle_inputs(spec, meta, args.seed)
+    budget = max(1.0, 20.0 / max(1, args.steps + args.warmup))
+
+    def one_seq(b):
+        r0, r1 = int(meta.cu_rows[b]), int(meta.cu_rows[b + 1])
+        O.layer_step(spec.shape, kb, vb, 0, xb[r0:r1], wb, meta.positions[r0:r1],
+                     meta.slots[r0:r1], np.array([0, r1 - r0], np.int32), meta.seq_lens[b:b + 1],
+                     meta.block_table[b:b + 1], meta.view[r0:r1])
+        return r1 - r0
+
+    # calibrate the sample on the first warm-up step
+    t0 = time.perf_counter()
+    one_seq(0)
+    per_seq = time.perf_counter() - t0
+    n_s = int(max(1, min(meta.batch, budget // max(per_seq, 1e-6))))
+    rows = int(meta.cu_rows[n_s] - meta.cu_rows[0])
+    times = []
     for i in range(args.warmup + args.steps):
-        v, desc, threads = oracle_sample(spec, meta, args.seed, budget_s=budget)
+        t0 = time.perf_counter()
+        for b in range(n_s):
+            one_seq(b)
+        dt = time.perf_counter() - t0
         if i >= args.warmup:
-            vals.append(v)
-    value = float(np.mean(vals))
-    R = meta.total_rows * spec.shape.n_layers
+            times.append(dt)
+    ms = 1000.0 * float(np.mean(times))
+    value = rows / (ms / 1000.0)
+    desc = (f"oracle (numpy float64) per step on the first {n_s} of {meta.batch} sequences of "
+            f"layer 0 ({rows} of {meta.total_rows} query rows), one sequence per call; "
+            f"{ms / 1000.0:.2f} s per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * R / value,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_block(spec, meta, args),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                         "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
     return 0
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([int(d.get("num_threads", 1)) for d in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
 
 
 def config_block(spec, meta, args):
@@ -438,6 +591,85 @@ def config_block(spec, meta, args):
             "page_size": sh.page_size, "track_k": meta.track_k,
             "l2": "flushed between timed steps (256 MB write)", "parallelism": f"replicas x{args.gpus}",
             "seed": args.seed}
+
+
+def roofline_of(spec, meta, kern_s, peaks, peak_src, kernel_name, traffic=None):
+    """Roofline of one layer step: the slower of algorithmic bytes over the
+    measured HBM copy rate and algorithmic FLOPs over the measured (burst)
+    bf16 rate, against the measured time of one layer step."""
+    byt, fl = W.algorithmic_bytes_flops(spec, meta)
+    t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
+    t_tc = fl / (peaks["bf16_tflops"] * 1e12)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    if bound == "tensor":
+        achieved, peak, unit = fl / kern_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = byt / kern_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic, "peak_source": f"{peak_src} (burst)", "kernel": kernel_name,
+            "kernel_us": kern_s * 1e6, "algorithmic_bytes": byt, "algorithmic_flops": fl,
+            "hbm_gbs_achieved": byt / kern_s / 1e9,
+            "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline": max(t_hbm, t_tc) / kern_s}
+
+
+def time_steps(step_fn, steps, warmup, flush, ev_layers=True):
+    """Runs `warmup` untimed steps, then `steps` steps bracketed by CUDA
+    events on the current stream with an L2 flush between them (outside the
+    events). step_fn(ev) runs one step and returns its kernel launches; with
+    ev = (start, end) it records them around its first-layer step and last
+    layer step. Returns (per-step ms list, per-step layer-span ms list,
+    launches)."""
+    for _ in range(warmup):
+        step_fn(None)
+    torch.cuda.synchronize()
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_ls = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev_le = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    launches = 0
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev_s[i].record()
+        launches += step_fn((ev_ls[i], ev_le[i]) if ev_layers else None)
+        ev_e[i].record()
+    torch.cuda.synchronize()
+    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(steps)]
+    layer_ms = [ev_ls[i].elapsed_time(ev_le[i]) for i in range(steps)] if ev_layers else step_ms
+    return step_ms, layer_ms, launches
+
+
+def measure_workload(name, seed, dev, steps, warmup, flush, peaks, peak_src, cpu_budget):
+    """Device-timed throughput of one layer workload plus its roofline and
+    an oracle CPU sample (for the per-workload table of the default run)."""
+    wl = Workload(name, seed, dev)
+    spec, meta = wl.spec, wl.meta
+    step_ms, layer_ms, launches = time_steps(lambda ev: wl.step(ev=ev, layer_span=True), steps,
+                                             warmup, flush)
+    wl.cache.check()
+    nl = spec.shape.n_layers
+    ms = float(np.mean(step_ms))
+    kern_s = float(np.mean(layer_ms)) / nl / 1000.0
+    roof = roofline_of(spec, meta, kern_s, peaks, peak_src,
+                       "fdllm_layer_step (fused step kernel + mass reduce), mean over layers")
+    cpu = None
+    if cpu_budget > 0:
+        v, desc, threads = oracle_sample(spec, meta, seed, budget_s=cpu_budget)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+    res = {"value": meta.total_rows / (ms / 1000.0), "unit": UNIT,
+           "layer_steps_per_s": nl / (ms / 1000.0), "ms_per_step": ms, "steps": steps,
+           "dtype": spec.shape.dtype, "gpu_launches": launches,
+           "config": config_block(spec, meta, argparse.Namespace(gpus=1, seed=seed)),
+           "roofline": {k: roof[k] for k in ("bound", "achieved", "peak", "unit", "frac", "kernel_us",
+                                              "roofline_us", "algorithmic_bytes",
+                                              "algorithmic_flops")},
+           "cpu_baseline": cpu}
+    wl.cache.close()
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
+PER_WORKLOAD = ("tiny_f32", "llada8b_b1", "two_view_b8", "stacked32_b4")
 
 
 def run_native(args):
@@ -463,20 +695,10 @@ def run_native(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_ls = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev_le = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    launches = 0
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        ev_s[i].record()
-        launches += wl.step(ev=(ev_ls[i], ev_le[i]))
-        ev_e[i].record()
-    torch.cuda.synchronize()
+    step_ms, layer_ms, launches = time_steps(lambda ev: wl.step(ev=ev), args.steps, 0, flush)
     barrier()
     t_wall1 = time.time()
     if sampler:
@@ -484,38 +706,36 @@ def run_native(args):
         time.sleep(0.25)
         sampler.stop()
     wl.cache.check()
-    step_ms = [ev_s[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
-    layer_ms = [ev_ls[i].elapsed_time(ev_le[i]) for i in range(args.steps)]
     total_ms_local = float(sum(step_ms))
     total_ms, _, value = aggregate(total_ms_local, meta.total_rows * args.steps, dev)
 
     # roofline of the dominant kernel (the fused layer step, layer 0)
-    byt, fl = W.algorithmic_bytes_flops(spec, meta)
     kern_s = float(np.mean(layer_ms)) / 1000.0
-    t_hbm = byt / (peaks["hbm_gbs"] * 1e9)
-    t_tc = fl / (peaks["bf16_tflops"] * 1e12)
-    bound = "tensor" if t_tc >= t_hbm else "hbm"
-    if bound == "tensor":
-        achieved, peak, unit = fl / kern_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    else:
-        achieved, peak, unit = byt / kern_s / 1e9, peaks["hbm_gbs"], "GB/s"
     traffic = args.traffic if args.traffic is not None else captured_traffic(spec.name)
-    roof = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-            "traffic": traffic, "peak_source": f"{peak_src} (burst)",
-            "kernel": "fdllm_layer_step (fused step kernel + mass reduce), layer 0",
-            "kernel_us": kern_s * 1e6, "algorithmic_bytes": byt, "algorithmic_flops": fl,
-            "hbm_gbs_achieved": byt / kern_s / 1e9,
-            "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline": max(t_hbm, t_tc) / kern_s}
+    roof = roofline_of(spec, meta, kern_s, peaks, peak_src,
+                       "fdllm_layer_step (fused step kernel + mass reduce), layer 0", traffic)
+    if traffic is not None:
+        roof["traffic_source"] = CAPTURED_TRAFFIC[spec.name]["source"]
 
     e2e_ms, serial_ms, h2d, d2h = e2e_measure(wl, max(10, min(args.steps, 200)))
     e2e_ms_max = reduce_max(e2e_ms, dev)
     serial_ms_max = reduce_max(serial_ms, dev)
     e2e_value = meta.total_rows * world / (e2e_ms_max / 1000.0)
+    wl.cache.close()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, threads = oracle_sample(spec, meta, args.seed + rank)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    # the other layer workloads, each device-timed with its own roofline and
+    # oracle sample (single-GPU runs of the default workload only)
+    per = None
+    if world == 1 and not args.no_per_workload and args.workload == "b32_divergent":
+        per = {}
+        for name in PER_WORKLOAD:
+            per[name] = measure_workload(name, args.seed, dev, min(args.steps, 20), 3, flush, peaks,
+                                         peak_src, 0.0 if args.no_cpu_baseline else 4.0)
 
     clocks = sampler.summary() if sampler else None
     line = {
@@ -531,12 +751,74 @@ def run_native(args):
                 "serial_ms_per_step": serial_ms_max},
         "gpu_launches": launches, "clocks": clocks,
     }
+    if per is not None:
+        line["per_workload"] = per
     if rank == 0:
         print(json.dumps(line))
-    wl.cache.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+    return 0
+
+
+def run_unfused(args):
+    """The unfused PyTorch arm (the pages' prior art) on a layer workload:
+    same inputs and metric; printed as one JSON line with impl "unfused"."""
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    torch.backends.cuda.matmul.allow_tf32 = True
+    peaks, peak_src = load_peaks()
+    spec = W.get_spec(args.workload)
+    if spec.shape.dtype != "bf16":
+        print(json.dumps({"impl": "unfused", "unavailable": "the unfused arm serves bf16 workloads"}))
+        return 0
+    meta = W.make_meta(spec, args.seed + rank)
+    sh = spec.shape
+    nl = sh.n_layers
+    xs = [W.make_x(spec, meta, args.seed + rank, layer=l, device=dev) for l in range(nl)]
+    ws = [W.make_w(spec, args.seed + rank, layer=l, device=dev) for l in range(nl)]
+    kp, vp = W.make_pools(spec, meta, args.seed + rank, device=dev)
+    u = UnfusedStep(spec, meta, dev)
+    pos = torch.from_numpy(meta.positions).to(dev)
+    slots = torch.from_numpy(meta.slots).to(dev)
+    view = torch.from_numpy(meta.view).to(dev)
+    bt = torch.from_numpy(meta.block_table).to(dev)
+    out = torch.empty(meta.total_rows, sh.hidden, dtype=torch.float32, device=dev)
+    mass = torch.empty(meta.batch, meta.max_blocks * sh.page_size, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        for l in range(nl):
+            if ev is not None and l == 0:
+                ev[0].record()
+            u.step(l, kp, vp, xs[l], ws[l], pos, slots, view, bt, out, mass)
+            if ev is not None and l == nl - 1:
+                ev[1].record()
+        return 0
+
+    # kernels per step, counted once with the profiler (untimed)
+    step(None)
+    torch.cuda.synchronize()
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step(None)
+        torch.cuda.synchronize()
+    per_step = sum(1 for e in prof.events() if e.device_type.name == "CUDA")
+    step_ms, layer_ms, _ = time_steps(step, args.steps, args.warmup, flush)
+    ms = float(np.mean(step_ms))
+    roof = roofline_of(spec, meta, float(np.mean(layer_ms)) / nl / 1000.0, peaks, peak_src,
+                       "unfused PyTorch layer step (all its kernels), mean over layers")
+    line = {"impl": "unfused", "metric": METRIC, "value": meta.total_rows / (ms / 1000.0),
+            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": config_block(spec, meta, argparse.Namespace(gpus=1, seed=args.seed)),
+            "layer_steps_per_s": nl / (ms / 1000.0), "roofline": roof,
+            "gpu_launches": per_step * args.steps,
+            "note": "torch/cuBLAS kernels, not this library's; selection not included"}
+    if rank == 0:
+        print(json.dumps(line))
     return 0
 
 
@@ -876,11 +1158,13 @@ def main(argv=None):
     ap.add_argument("--workload", default="b32_divergent",
                     choices=sorted(W.WORKLOADS) + sorted(W.VERIFY_WORKLOADS) +
                     sorted(W.OPROJ_WORKLOADS))
-    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--impl", default="native", choices=["native", "reference", "unfused"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the step kernel, when captured for this build")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the table of the other layer workloads in the default run")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -890,6 +1174,8 @@ def main(argv=None):
         return run_oproj(args)
     if args.impl == "reference":
         return run_reference(args)
+    if args.impl == "unfused":
+        return run_unfused(args)
     return run_native(args)
 
 

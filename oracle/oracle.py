@@ -144,7 +144,7 @@ def visible_keys(L: int, view: np.ndarray, positions: np.ndarray, slots: np.ndar
 # --------------------------------------------------------------------------
 
 def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
-               cu_rows, seq_lens, block_table, view, probs=None):
+               cu_rows, seq_lens, block_table, view, probs=None, accumulate="f64"):
     """One Flash-Cache + scheduled-attention layer step.
 
     shape: object with dtype ("bf16"/"f32"), hidden, n_heads, head_dim,
@@ -166,8 +166,19 @@ def layer_step(shape, k_pool, v_pool, layer, x_bits, w_bits, positions, slots,
     block table. [FD ¶2]: the step's rows are the unmasking window plus the
     tracked tokens; the per-key attention mass feeds the next tracked set.
     [FD ¶3]: the draft and mask views share positions (hence RoPE) and are
-    isolated from each other."""
-    a = project(shape, x_bits, w_bits)
+    isolated from each other.
+
+    accumulate: "f64" (default) takes the projection exactly (float64 sums
+    of exact products); "f32" takes it from a float32 matrix product of the
+    same bf16/fp32 inputs (project_f32acc): the bf16-in / fp32-accumulate
+    reading of the step, whose fresh k and v can land on the other side of a
+    bf16 rounding midpoint. Everything after the projection is the same."""
+    if accumulate == "f64":
+        a = project(shape, x_bits, w_bits)
+    elif accumulate == "f32":
+        a = project_f32acc(shape, x_bits, w_bits)
+    else:
+        raise ValueError(f"accumulate must be 'f64' or 'f32', got {accumulate!r}")
     return layer_step_from_projection(shape, k_pool, v_pool, layer, a, positions, slots,
                                       cu_rows, seq_lens, block_table, view, probs)
 
@@ -176,6 +187,16 @@ def project(shape, x_bits, w_bits):
     """Step 1, the QKV projection: a = x Wqkv in float64 (library matmul on
     the exact values of the bf16/fp32 inputs). [R, 3H]."""
     return decode(x_bits, shape.dtype) @ decode(w_bits, shape.dtype)
+
+
+def project_f32acc(shape, x_bits, w_bits):
+    """Step 1 with float32 accumulation: the library's float32 matrix
+    product of the same inputs (each bf16/fp32 input is exact in float32),
+    returned as float64. It differs from `project` only by float32 rounding
+    of the sums (at most about K * 2^-24 * sum |x_k w_k| per entry)."""
+    xf = decode(x_bits, shape.dtype).astype(np.float32)
+    wf = decode(w_bits, shape.dtype).astype(np.float32)
+    return (xf @ wf).astype(np.float64)
 
 
 def layer_step_from_projection(shape, k_pool, v_pool, layer, a, positions, slots, cu_rows,

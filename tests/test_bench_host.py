@@ -21,16 +21,30 @@ def test_captured_traffic_needs_matching_sources(tmp_path, monkeypatch):
     root = tmp_path
     csrc = root / "kv_cache_attention_flash_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (root / "profiles").mkdir()
     for name, body in (("step_bf16.cu", "int a;\n"), ("ptx.cuh", "int b;\n"), ("api.cu", "int c;\n")):
         (csrc / name).write_text(body)
-    hashes = " ".join(bench.code_hash(str(csrc / n)) for n in ("step_bf16.cu", "ptx.cuh", "api.cu"))
-    (root / "profiles" / "step_bf16_demo.md").write_text(
-        f"notes\n\ntraffic_bytes_per_launch: 12345\nkernel_sources_sha256: {hashes}\n")
+    hashes = [bench.code_hash(str(csrc / n)) for n in ("step_bf16.cu", "ptx.cuh", "api.cu")]
     monkeypatch.setattr(bench, "ROOT", str(root))
+    monkeypatch.setattr(bench, "CAPTURED_TRAFFIC",
+                        {"demo": {"bytes": 12345.0, "sources": hashes, "source": "test"}})
     assert bench.captured_traffic("demo") == 12345.0
     (csrc / "api.cu").write_text("int c;  // same code, new comment\n")
     assert bench.captured_traffic("demo") == 12345.0
     (csrc / "api.cu").write_text("int c2;\n")
     assert bench.captured_traffic("demo") is None
     assert bench.captured_traffic("missing") is None
+
+
+def test_reference_arm_times_whole_sampled_steps(capsys):
+    """The reference arm's ms_per_step is the measured time of its sampled
+    steps, so ms_per_step x steps fits the run."""
+    import json
+    import time
+    t0 = time.time()
+    assert bench.main(["--impl", "reference", "--workload", "tiny_f32", "--steps", "3",
+                       "--warmup", "3"]) == 0
+    wall = time.time() - t0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["ms_per_step"] * line["steps"] / 1000.0 <= wall
+    assert line["cpu_baseline"]["kind"] == "oracle"

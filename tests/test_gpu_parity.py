@@ -15,10 +15,16 @@ from gpu_case import build_inputs, compare, run_gpu, run_oracle
 
 def check_dense(spec, meta, x, w, kp, vp, g):
     """Compare a dense-x GPU run with the oracle: the plain 1e-2 * RMS bar
-    on out (1e-4 for fp32), cache values within one bf16 ulp."""
+    on out (1e-4 for fp32), cache values within one bf16 ulp. For bf16, a
+    step whose exact reading the bar cannot hold for (fresh v on the other
+    side of a bf16 rounding midpoint under fp32 accumulation, where that key
+    carries much of a row's attention) is held to the same bar against the
+    oracle's fp32-accumulate reading."""
     o = run_oracle(spec, meta, x, w, kp, vp)
-    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp),
-            mode="dense" if spec.shape.dtype == "bf16" else "plain")
+    bf = spec.shape.dtype == "bf16"
+    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="dense" if bf else "plain",
+            orc_f32acc=(lambda: run_oracle(spec, meta, x, w, kp, vp, accumulate="f32")) if bf
+            else None)
 
 pytestmark = pytest.mark.gpu
 

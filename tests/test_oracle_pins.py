@@ -135,7 +135,8 @@ def run_oracle(shape, c, **over):
     d = dict(c)
     d.update(over)
     return O.layer_step(shape, d["kp"], d["vp"], 0, d["x"], d["w"], d["positions"], d["slots"],
-                        d["cu"], d["lens"], d["bt"], d["view"])
+                        d["cu"], d["lens"], d["bt"], d["view"],
+                        accumulate=d.get("accumulate", "f64"))
 
 
 def brute_force(shape, c):
@@ -292,6 +293,52 @@ def test_softmax_rows_sum_to_one_and_match_library():
     assert np.all(P[~vis] == 0)
     ref = torch.softmax(torch.from_numpy(np.where(vis, S, -np.inf)[1:]), dim=-1).numpy()
     assert np.allclose(P[1:], ref, rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# the float32-accumulation reading of the projection
+# --------------------------------------------------------------------------
+
+
+def test_f32_accumulated_projection_is_within_the_float32_bound():
+    """project_f32acc differs from the exact projection by no more than the
+    standard bound for a float32 sum of K exact products, K * 2^-24 *
+    sum_k |x_k w_k| (any summation order), and it does differ somewhere."""
+    sh = Shape("bf16", 512, 4, 128, 64, 1e4)
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((40, 512))).astype(np.float32)
+    w = (rng.standard_normal((512, 1536)) * 0.02).astype(np.float32)
+    xb = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    wb = torch.from_numpy(w).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    xv = torch_bf16_value(xb).numpy()
+    wv = torch_bf16_value(wb).numpy()
+    exact = xv @ wv                                # products of 8-bit significands are exact
+    a32 = O.project_f32acc(sh, xb, wb)
+    bound = 512 * 2.0 ** -24 * (np.abs(xv) @ np.abs(wv))
+    assert np.all(np.abs(a32 - exact) <= bound)
+    assert np.any(a32 != exact)
+    assert np.allclose(O.project(sh, xb, wb), exact, rtol=0, atol=1e-12)
+
+
+def test_f32_reading_equals_exact_reading_for_one_hot_rows():
+    """With one-hot x (a power of two times one weight row) every projected
+    value is exact in float32 too, so both readings give identical steps."""
+    sh = SHAPES["bf16"]
+    rng = np.random.default_rng(22)
+    c = make_case(rng, sh, lens=[30, 41], rows_per_seq=[6, 9])
+    R = c["x"].shape[0]
+    onehot = np.zeros((R, sh.hidden), np.float32)
+    onehot[np.arange(R), rng.integers(0, sh.hidden, R)] = 64.0
+    c["x"] = torch.from_numpy(onehot).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    o64 = run_oracle(sh, c)
+    o32 = run_oracle(sh, c, accumulate="f32")
+    for a, b in zip(o64, o32):
+        assert np.array_equal(a, b)
+    # dense rows: the readings stay close
+    c2 = make_case(rng, sh, lens=[30, 41], rows_per_seq=[6, 9])
+    d64 = run_oracle(sh, c2)[0]
+    d32 = run_oracle(sh, c2, accumulate="f32")[0]
+    assert np.max(np.abs(d64 - d32)) <= 1e-2 * np.sqrt(np.mean(d64 ** 2))
 
 
 # --------------------------------------------------------------------------

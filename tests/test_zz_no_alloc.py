@@ -126,8 +126,13 @@ def test_noalloc_matches_layer_step_twice(name):
                            meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table, meta.view)
         tracked = fd.fdllm_select_tracked(mass_b, sl_d, meta.track_k, ecu_d, esl_d).cpu().numpy()
         g = GpuResult(out_b.cpu().numpy(), mass_b.cpu().numpy(), tracked, bits(kb), bits(vb))
+        def f32acc(kb_=o_kp, vb_=o_vp, x_=x):
+            return O.layer_step(sh, kb_, vb_, 0, W.bits_np(x_), W.bits_np(w), meta.positions,
+                                meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table,
+                                meta.view, accumulate="f32")
         compare(spec, meta, g, orc, o_kp, o_vp, mode="dense" if sh.dtype == "bf16" else "plain",
-                label=f"{name} no-alloc call {call + 1}")
+                label=f"{name} no-alloc call {call + 1}",
+                orc_f32acc=f32acc if sh.dtype == "bf16" else None)
         o_kp, o_vp = orc[2], orc[3]
     cache.close()
 
