@@ -218,6 +218,17 @@ class Workload:
         R = m.total_rows
         H = sh.hidden
         self.out = torch.empty(R, H, dtype=torch.float32, device=device)
+        # a chained stack: x_0 only; layer l's x is the residual stream
+        # x_{l-1} + out_{l-1} W_o,{l-1} (bf16 out, output projection with the
+        # residual), kept in self.xs while x_0 stays as drawn
+        self.chained = self.spec.chained
+        if self.chained:
+            from kv_cache_attention_flash_b200.stack import LayerStack
+            self.x = self.x[:1]
+            self.w_o = [W.make_w_o(self.spec, seed, layer=l, device=device)
+                        for l in range(self.n_layers)]
+            self.stack = LayerStack(self.cache, self.w, self.w_o)
+            self.xs = torch.empty_like(self.x[0])
         self.mass = torch.empty(m.batch, m.max_blocks * sh.page_size, dtype=torch.float32, device=device)
         self.tracked = torch.empty(m.batch, m.track_k, dtype=torch.int32, device=device)
         self.launches_per_step = None
@@ -231,6 +242,17 @@ class Workload:
         n = 0
         xs = x_list if x_list is not None else self.x
         nl = self.n_layers
+        if self.chained:
+            if ev is not None:
+                ev[0].record()
+            self.stack.run(m.cu_rows, m.seq_lens, xs[0], self.pos, self.bt, self.view, self.slots,
+                           self.mass, x_out=self.xs)
+            n += self.stack.launches
+            if ev is not None:
+                ev[1].record()
+            fd.fdllm_select_tracked(self.mass, self.seq_lens_d, m.track_k, self.ex_cu, self.ex_sl,
+                                    self.tracked)
+            return n + fd.fdllm_last_launch_count()
         for l in range(nl):
             if ev is not None and l == 0:
                 ev[0].record()
@@ -435,13 +457,15 @@ def e2e_measure(wl: Workload, steps: int):
     dmeta0 = (wl.pos, wl.slots, wl.view, wl.bt)
     hmeta = [t.cpu().pin_memory() for t in dmeta0]
     bufs = []
+    # a chained stack's result is the final residual stream (bf16)
+    res_like = wl.xs if wl.chained else wl.out
     for _ in range(NB):
         bufs.append({
             "x": [torch.empty_like(x) for x in wl.x],
             "meta": [torch.empty_like(t) for t in dmeta0],
-            "out": torch.empty_like(wl.out), "mass": torch.empty_like(wl.mass),
+            "out": torch.empty_like(res_like), "mass": torch.empty_like(wl.mass),
             "tr": torch.empty_like(wl.tracked),
-            "hout": torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory(),
+            "hout": torch.empty(res_like.shape, dtype=res_like.dtype).pin_memory(),
             "hmass": torch.empty(wl.mass.shape, dtype=wl.mass.dtype).pin_memory(),
             "htr": torch.empty(wl.tracked.shape, dtype=wl.tracked.dtype).pin_memory(),
             "ev_in": torch.cuda.Event(), "ev_comp": torch.cuda.Event(), "ev_out": torch.cuda.Event(),
@@ -456,6 +480,12 @@ def e2e_measure(wl: Workload, steps: int):
 
     def compute(b, stream):
         pos, slots, view, bt = b["meta"]
+        if wl.chained:
+            wl.stack.run(m.cu_rows, m.seq_lens, b["x"][0], pos, bt, view, slots, b["mass"],
+                         stream=stream, x_out=b["out"])
+            fd.fdllm_select_tracked(b["mass"], wl.seq_lens_d, m.track_k, wl.ex_cu, wl.ex_sl,
+                                    b["tr"], stream=stream)
+            return
         for l in range(wl.n_layers):
             fd.fdllm_layer_step(wl.cache.handle, l, m.cu_rows, m.seq_lens, m.max_blocks, b["x"][l],
                                 wl.w[l], pos, bt, view, b["out"], b["mass"], slots, stream=stream)
@@ -464,7 +494,7 @@ def e2e_measure(wl: Workload, steps: int):
 
     def one_serial():
         b = bufs[0]
-        for l in range(wl.n_layers):
+        for l in range(len(wl.x)):
             b["x"][l].copy_(hx[l], non_blocking=True)
         for d, h in zip(b["meta"], hmeta):
             d.copy_(h, non_blocking=True)
@@ -478,7 +508,7 @@ def e2e_measure(wl: Workload, steps: int):
         if i >= NB:   # step i-NB no longer reads these inputs
             s_in.wait_event(b["ev_comp"])
         with torch.cuda.stream(s_in):
-            for l in range(wl.n_layers):
+            for l in range(len(wl.x)):
                 b["x"][l].copy_(hx[l], non_blocking=True)
             for d, h in zip(b["meta"], hmeta):
                 d.copy_(h, non_blocking=True)
@@ -669,7 +699,7 @@ def measure_workload(name, seed, dev, steps, warmup, flush, peaks, peak_src, cpu
     return res
 
 
-PER_WORKLOAD = ("tiny_f32", "llada8b_b1", "two_view_b8", "stacked32_b4")
+PER_WORKLOAD = ("tiny_f32", "llada8b_b1", "two_view_b8", "stacked32_b4", "stacked32_b4_chained")
 
 
 def run_native(args):
@@ -1150,6 +1180,63 @@ def run_oproj(args):
     return 0
 
 
+DECODE_METRIC = "toy decode loop: decoded tokens/s (random weights; throughput only)"
+DECODE_CONFIGS = {
+    # LLaDA-8B layer shape, 4 chained layers, batch 8, 256-token prompt and
+    # 256-token generation, 32-token window, 32 tracked tokens
+    "decode_llada8b_4l": dict(hidden=4096, n_heads=32, head_dim=128, n_layers=4, batch=8,
+                              prompt_len=256, gen_len=256, window=32, track_k=32, tau=0.5),
+}
+
+
+def run_decode(args):
+    """The toy decode loop (kv_cache_attention_flash_b200.decode_loop): a
+    chunked prefill, then decode steps until `steps` steps are timed (or
+    every sequence finished). Timed with CUDA events around each step; the
+    host work between steps (acceptance, next rows) is inside the timed
+    span, as in a serving loop."""
+    from kv_cache_attention_flash_b200.decode_loop import ToyDecodeLoop
+    from kv_cache_attention_flash_b200.workloads import ToyConfig
+    rank, world, local = dist_env()
+    if args.impl != "native":
+        print(json.dumps({"impl": args.impl, "unavailable": "the toy decode loop has one arm"}))
+        return 0
+    if world > 1:
+        torch.cuda.set_device(local)
+    cfg = ToyConfig(seed=args.seed + rank, **DECODE_CONFIGS[args.workload])
+    loop = ToyDecodeLoop(cfg, "cuda")
+    loop.prefill()
+    for _ in range(args.warmup):
+        loop.step()
+    torch.cuda.synchronize()
+    accepted, rows, times = 0, 0, []
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.steps):
+        if loop.done():
+            break
+        r0 = loop.rows_done
+        e0.record()
+        acc, _, _ = loop.step()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        accepted += int(acc.sum())
+        rows += loop.rows_done - r0
+    loop.cache.check()
+    ms = float(np.mean(times))
+    n = len(times)
+    line = {"metric": DECODE_METRIC, "value": accepted / (sum(times) / 1000.0), "unit": "tokens/s",
+            "n_gpus": 1, "steps": n, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic (random weights)",
+            "config": {"workload": args.workload, **DECODE_CONFIGS[args.workload]},
+            "query_rows_per_s": rows / (sum(times) / 1000.0),
+            "accepted_per_step": accepted / max(n, 1)}
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1157,7 +1244,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="b32_divergent",
                     choices=sorted(W.WORKLOADS) + sorted(W.VERIFY_WORKLOADS) +
-                    sorted(W.OPROJ_WORKLOADS))
+                    sorted(W.OPROJ_WORKLOADS) + sorted(DECODE_CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference", "unfused"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--traffic", type=float, default=None,
@@ -1172,6 +1259,8 @@ def main(argv=None):
         return run_verify(args)
     if args.workload in W.OPROJ_WORKLOADS:
         return run_oproj(args)
+    if args.workload in DECODE_CONFIGS:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.impl == "unfused":

@@ -285,25 +285,33 @@ FDLLM_API fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_
                                       int32_t n_heads, int32_t n_bins, int32_t* bin_start,
                                       int32_t* tiles);
 
-/* Output projection of the attention block: y = attn_out W_o, bf16 in and
- * out, fp32 accumulation (one tcgen05 GEMM launch).
+/* Output projection of the attention block: y = residual + attn_out W_o,
+ * bf16 in and out, fp32 accumulation (one tcgen05 GEMM launch).
  * [FD] paragraph 1 covers a layer up to the attention output; the
  * projection after it is the plain linear map over the heads' outputs side
  * by side, read with the conventions of wqkv (y = x W, row-major, no bias).
+ * With a residual it closes the layer's attention sub-block as a
+ * transformer's residual stream does (x_next = x + attn_out W_o), which is
+ * how a stack of layer steps chains one layer's output into the next
+ * layer's x.
  *   attn_out: DEVICE bf16 [rows][hidden], e.g. fdllm_layer_step's out with
- *     step->out_bf16 = 1.
- *   w_o: DEVICE bf16 [hidden][hidden], row-major.
- *   y: DEVICE bf16 [rows][hidden] out, each value rounded to nearest even
- *     from the fp32 sum; must not overlap the inputs.
+ *     step->out_bf16 = 1. Must not overlap y.
+ *   w_o: DEVICE bf16 [hidden][hidden], row-major. Must not overlap y.
+ *   residual: DEVICE bf16 [rows][hidden] or NULL (no residual). It may be y
+ *     itself (an in-place update of the residual stream), but may not
+ *     overlap y otherwise.
+ *   y: DEVICE bf16 [rows][hidden] out; each value is the fp32 sum
+ *     (accumulator + residual) rounded once to nearest even.
  *   rows >= 0 (0 enqueues nothing); hidden a positive multiple of 256.
- *   All three pointers 16-byte aligned.
+ *   All pointers 16-byte aligned.
  *   status: DEVICE int32 or NULL; a bounded in-kernel wait that gives up
  *     writes FDLLM_ERR_TIMEOUT there (and y is then incomplete); nothing
  *     else writes it.
  * Host-detectable errors return FDLLM_ERR_INVALID_ARG or
  * FDLLM_ERR_UNSUPPORTED and enqueue nothing. */
-FDLLM_API fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t rows,
-                                   int32_t hidden, int32_t* status, void* stream);
+FDLLM_API fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, const void* residual,
+                                   void* y, int32_t rows, int32_t hidden, int32_t* status,
+                                   void* stream);
 
 /* Synchronises `stream`, reads and clears the handle's device error word.
  * Returns FDLLM_OK, FDLLM_ERR_DEVICE_BOUNDS, FDLLM_ERR_TIMEOUT or

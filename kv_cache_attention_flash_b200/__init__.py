@@ -215,19 +215,23 @@ def fdllm_plan_tile_schedule(group_cost: Sequence[float], n_heads: int, n_bins: 
 
 
 def fdllm_oproj(attn_out: torch.Tensor, w_o: torch.Tensor, y: Optional[torch.Tensor] = None,
-                status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Output projection y = attn_out W_o (see include/fdllm.h): bf16
-    [rows, hidden] times bf16 [hidden, hidden], bf16 result."""
+                status: Optional[torch.Tensor] = None, stream=None,
+                residual: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Output projection y = residual + attn_out W_o (see include/fdllm.h):
+    bf16 [rows, hidden] times bf16 [hidden, hidden], bf16 result; residual
+    is optional and may be y itself."""
     lib = load()
     rows, hidden = attn_out.shape
     if tuple(w_o.shape) != (hidden, hidden):
         raise ValueError(f"w_o must be [{hidden}, {hidden}], got {tuple(w_o.shape)}")
+    if residual is not None and tuple(residual.shape) != (rows, hidden):
+        raise ValueError(f"residual must be [{rows}, {hidden}], got {tuple(residual.shape)}")
     if y is None:
         y = torch.empty(rows, hidden, dtype=torch.bfloat16, device=attn_out.device)
     check_status(lib.fdllm_oproj(
         _dev_ptr(attn_out, torch.bfloat16, "attn_out"), _dev_ptr(w_o, torch.bfloat16, "w_o"),
-        _dev_ptr(y, torch.bfloat16, "y"), int(rows), int(hidden),
-        _dev_ptr(status, torch.int32, "status"), _stream_ptr(stream)))
+        _dev_ptr(residual, torch.bfloat16, "residual"), _dev_ptr(y, torch.bfloat16, "y"),
+        int(rows), int(hidden), _dev_ptr(status, torch.int32, "status"), _stream_ptr(stream)))
     return y
 
 

@@ -54,7 +54,7 @@ SIGNATURES = {
     "fdllm_verify_accept": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _vp, ctypes.c_float, _vp,
                                    _vp, _vp, _vp]),
     "fdllm_plan_tile_schedule": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
-    "fdllm_oproj": (_i32, [_vp, _vp, _vp, _i32, _i32, _vp, _vp]),
+    "fdllm_oproj": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp]),
     "fdllm_check": (_i32, [_vp, _vp]),
     "fdllm_inject_fault": (_i32, [_vp, _i32, ctypes.c_int64]),
     "fdllm_status_string": (ctypes.c_char_p, [_i32]),

@@ -826,8 +826,8 @@ fdllm_status fdllm_plan_tile_schedule(const double* group_cost, int32_t n_groups
   return FDLLM_OK;
 }
 
-fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t rows,
-                         int32_t hidden, int32_t* status, void* stream) {
+fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, const void* residual, void* y,
+                         int32_t rows, int32_t hidden, int32_t* status, void* stream) {
   NvtxRange nvtx_range("fdllm_oproj");
   if (rows < 0 || hidden <= 0)
     return fail(FDLLM_ERR_INVALID_ARG, "oproj: rows >= 0 and hidden > 0 required");
@@ -839,8 +839,21 @@ fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t
   }
   if (!attn_out || !w_o || !y) return fail(FDLLM_ERR_INVALID_ARG, "oproj: null pointer");
   if ((reinterpret_cast<uintptr_t>(attn_out) | reinterpret_cast<uintptr_t>(w_o) |
-       reinterpret_cast<uintptr_t>(y)) & 15)
+       reinterpret_cast<uintptr_t>(residual) | reinterpret_cast<uintptr_t>(y)) & 15)
     return fail(FDLLM_ERR_INVALID_ARG, "oproj: pointers must be 16-byte aligned");
+  {
+    // y may be the residual itself, but overlaps no input otherwise
+    const uintptr_t yb = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t ye = yb + (uintptr_t)rows * hidden * 2;
+    auto overlaps = [&](const void* p, size_t bytes) {
+      const uintptr_t b = reinterpret_cast<uintptr_t>(p);
+      return b < ye && yb < b + bytes;
+    };
+    const size_t act = (size_t)rows * hidden * 2;
+    if (overlaps(attn_out, act) || overlaps(w_o, (size_t)hidden * hidden * 2) ||
+        (residual && residual != y && overlaps(residual, act)))
+      return fail(FDLLM_ERR_INVALID_ARG, "oproj: y overlaps an input");
+  }
   // Tile width: 256 columns unless 128-column tiles finish sooner. A
   // 128-wide tile does half the work but takes 0.87 of a 256-wide one's time
   // on B200 (26.6 vs 30.7 us at 1536 x 4096: the narrower MMA re-reads its A
@@ -855,7 +868,7 @@ fdllm_status fdllm_oproj(const void* attn_out, const void* w_o, void* y, int32_t
   if (!encode_bf16_2d(&to, attn_out, (uint64_t)rows, (uint64_t)hidden, 128u) ||
       !encode_w_3d(&tw, w_o, (uint64_t)hidden, (uint32_t)(bn / 64)))
     return fail(FDLLM_ERR_CUDA, "oproj: cuTensorMapEncodeTiled failed");
-  cudaError_t e = launch_oproj(&to, &tw, bn, y, rows, hidden, status,
+  cudaError_t e = launch_oproj(&to, &tw, bn, residual, y, rows, hidden, status,
                                reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "oproj: launch");
   g_last_launches = 1;

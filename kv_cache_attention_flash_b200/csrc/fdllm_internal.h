@@ -87,11 +87,12 @@ struct StepArgs {
 };
 
 // Launchers (return cudaGetLastError()).
-// y = o W_o in tiles of 128 rows x bn (256 or 128) columns: tmap_o over o
+// y = residual + o W_o (residual may be null or y itself) in tiles of 128
+// rows x bn (256 or 128) columns: tmap_o over o
 // [rows][hidden] with 128-row boxes, tmap_w the 3-D view of W_o {64 columns,
 // hidden K rows, hidden / 64 column blocks} with boxes of bn / 64 blocks.
-cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, void* y, int rows,
-                         int hidden, int32_t* status, cudaStream_t stream);
+cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, const void* residual,
+                         void* y, int rows, int hidden, int32_t* status, cudaStream_t stream);
 size_t oproj_smem_bytes();
 // tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
 // tmap_w1: the one-block view of Wqkv (box {64, 64, 2, 1, 1}), used when

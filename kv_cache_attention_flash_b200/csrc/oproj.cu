@@ -1,5 +1,6 @@
-// Output projection of the attention block: y = o W_o, bf16 operands, fp32
-// accumulation in TMEM, bf16 result.
+// Output projection of the attention block: y = residual + o W_o, bf16
+// operands, fp32 accumulation in TMEM (the residual added in fp32), one
+// rounding to bf16.
 //
 // "Flash-dLLM: I/O-Aware KV Caching and Parallel Decoding for Fast,
 // Memory-Efficient Diffusion LLMs" (ai4snews summary), paragraph 1, covers a
@@ -16,8 +17,9 @@
 //     ring of 192 KB (4 stages of 48 KB, or 6 of 32 KB).
 //   warp 1 (lane 0): tcgen05.mma issuer (M128 N-BN K16, A K-major, B
 //     N-major) into BN TMEM columns; owns the TMEM allocation.
-//   warps 2-5: epilogue, one TMEM lane quadrant each: fp32 accumulator ->
-//     bf16 (round to nearest even) -> 16-byte stores of y.
+//   warps 2-5: epilogue, one TMEM lane quadrant each: fp32 accumulator
+//     (+ the residual row, read before the store so that y may be the
+//     residual) -> bf16 (round to nearest even) -> 16-byte stores of y.
 // All waits are bounded; a timeout writes FDLLM_ERR_TIMEOUT to the caller's
 // status word (if given), stops the ring, drains the copies already issued
 // and frees TMEM.
@@ -75,7 +77,8 @@ __device__ __forceinline__ bool op_wait(OpCtrl* c, uint64_t* bar, uint32_t parit
 template <int BN>
 __global__ void __launch_bounds__(OP_THREADS, 1)
     oproj_kernel(const __grid_constant__ CUtensorMap tmap_o, const __grid_constant__ CUtensorMap tmap_w,
-                 __nv_bfloat16* y, int rows, int hidden, int32_t* status) {
+                 const __nv_bfloat16* resid, __nv_bfloat16* y, int rows, int hidden,
+                 int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -169,6 +172,20 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
         ptx::tmem_ld32(taddr + c0, v);
         ptx::tmem_ld_wait();
         if (row < rows) {
+          if (resid) {   // read before the store: y may be the residual itself
+            const uint4* rsrc =
+                reinterpret_cast<const uint4*>(resid + (size_t)row * hidden + n0 + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 r4 = rsrc[q];
+              const uint32_t rw[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[8 * q + 2 * e] += __uint_as_float(rw[e] << 16);
+                v[8 * q + 2 * e + 1] += __uint_as_float(rw[e] & 0xffff0000u);
+              }
+            }
+          }
           uint4* dst = reinterpret_cast<uint4*>(yrow + c0);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -186,8 +203,8 @@ __global__ void __launch_bounds__(OP_THREADS, 1)
 }
 
 template <int BN>
-cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, void* y, int rows, int hidden,
-                            int32_t* status, cudaStream_t stream) {
+cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, const void* resid, void* y,
+                            int rows, int hidden, int32_t* status, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = opt_in_smem(reinterpret_cast<const void*>(oproj_kernel<BN>), OP_SMEM_BYTES,
                               attr_done);
@@ -195,7 +212,8 @@ cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, void* y, int
   dim3 grid((rows + OP_BM - 1) / OP_BM, hidden / BN);
   oproj_kernel<BN><<<grid, OP_THREADS, OP_SMEM_BYTES, stream>>>(
       *reinterpret_cast<const CUtensorMap*>(tmap_o), *reinterpret_cast<const CUtensorMap*>(tmap_w),
-      reinterpret_cast<__nv_bfloat16*>(y), rows, hidden, status);
+      reinterpret_cast<const __nv_bfloat16*>(resid), reinterpret_cast<__nv_bfloat16*>(y), rows,
+      hidden, status);
   return cudaGetLastError();
 }
 
@@ -203,11 +221,13 @@ cudaError_t launch_oproj_bn(const void* tmap_o, const void* tmap_w, void* y, int
 
 size_t oproj_smem_bytes() { return OP_SMEM_BYTES; }
 
-cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, void* y, int rows,
-                         int hidden, int32_t* status, cudaStream_t stream) {
+cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, const void* resid,
+                         void* y, int rows, int hidden, int32_t* status, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  if (bn == 256) return launch_oproj_bn<256>(tmap_o, tmap_w, y, rows, hidden, status, stream);
-  if (bn == 128) return launch_oproj_bn<128>(tmap_o, tmap_w, y, rows, hidden, status, stream);
+  if (bn == 256)
+    return launch_oproj_bn<256>(tmap_o, tmap_w, resid, y, rows, hidden, status, stream);
+  if (bn == 128)
+    return launch_oproj_bn<128>(tmap_o, tmap_w, resid, y, rows, hidden, status, stream);
   return cudaErrorInvalidValue;
 }
 

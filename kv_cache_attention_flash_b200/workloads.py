@@ -58,6 +58,9 @@ class WorkloadSpec:
     ctx_min: int = 0              # divergent: L_b ~ U[ctx_min, ctx_max]
     ctx_max: int = 0
     window: int = 32
+    # stack: layer l's x is the residual stream x_l + out_{l-1} W_o,{l-1}
+    # (chained), or an independent seeded draw per layer (not chained)
+    chained: bool = False
     tracked: int = 32             # tracked rows per update-stage sequence
     track_k: int = 32             # k of the next step's top-k selection
     view_rows: int = 32           # two_view: rows per view
@@ -86,6 +89,12 @@ WORKLOADS: Dict[str, WorkloadSpec] = {
     "stacked32_b4": WorkloadSpec("stacked32_b4", dataclasses.replace(LLADA8B, n_layers=32),
                                  batch=4, kind="window", ctx_len=8192, prompt_len=0,
                                  window=32, tracked=64, track_k=64),
+    # the same stack chained: each layer's bf16 out goes through its output
+    # projection into the residual stream that is the next layer's x
+    "stacked32_b4_chained": WorkloadSpec("stacked32_b4_chained",
+                                         dataclasses.replace(LLADA8B, n_layers=32), batch=4,
+                                         kind="window", ctx_len=8192, prompt_len=0, window=32,
+                                         tracked=64, track_k=64, chained=True),
 }
 
 # Small variants of the same structure (same code paths, oracle-sized).
@@ -97,6 +106,11 @@ SMALL_WORKLOADS: Dict[str, WorkloadSpec] = {
     "small_bf16_two_view": WorkloadSpec(
         "small_bf16_two_view", LayerShape("bf16", 512, 4, 128, 64, 10000.0),
         batch=3, kind="two_view", ctx_len=200, view_rows=24, track_k=8, spare_pages=2),
+    # a short chained stack at oracle size
+    "small_bf16_chained": WorkloadSpec(
+        "small_bf16_chained", LayerShape("bf16", 512, 4, 128, 64, 500000.0, n_layers=4),
+        batch=3, kind="window", ctx_len=300, prompt_len=64, window=16, tracked=16, track_k=8,
+        chained=True, spare_pages=2),
     "small_f32_divergent": WorkloadSpec(
         "small_f32_divergent", LayerShape("f32", 128, 2, 64, 16, 10000.0),
         batch=4, kind="divergent", ctx_min=20, ctx_max=90, window=8, tracked=8,
@@ -259,12 +273,40 @@ def make_x_onehot(spec: WorkloadSpec, meta: StepMeta, seed: int, scale: float = 
     return x.to(torch_dtype(spec.shape))
 
 
+def make_x_grid(spec: WorkloadSpec, meta: StepMeta, seed: int, layer: int = 0,
+                device="cpu") -> torch.Tensor:
+    """x [R, H] ~ N(0, 1) snapped to multiples of 1/4 in [-4, 4] (two-view:
+    mask rows share one vector, as in make_x). Together with make_w_grid
+    every product x_k W_kn is a multiple of 2^-12 and every partial sum of
+    4096 of them stays below 2^11 in magnitude, so each sum is exact in
+    float32 whatever the order of accumulation: the projection of these
+    dense, normally shaped inputs is exact in fp32 and fp64 alike."""
+    x = make_x(spec, meta, seed, layer=layer, device=device).float()
+    return (torch.clamp(torch.round(x * 4.0), -16, 16) / 4.0).to(torch_dtype(spec.shape))
+
+
+def make_w_grid(spec: WorkloadSpec, seed: int, layer: int = 0, device="cpu") -> torch.Tensor:
+    """Wqkv ~ N(0, 0.02^2) snapped to multiples of 2^-10 in [-127, 127] *
+    2^-10 (see make_x_grid)."""
+    w = make_w(spec, seed, layer=layer, device=device).float()
+    return (torch.clamp(torch.round(w * 1024.0), -127, 127) / 1024.0).to(torch_dtype(spec.shape))
+
+
 def make_w(spec: WorkloadSpec, seed: int, layer: int = 0, device="cpu") -> torch.Tensor:
     """Wqkv [H, 3H] row-major, N(0, 0.02^2); columns are [Q | K | V], each
     block head-major (head h at columns h*D .. h*D+D-1)."""
     H = spec.shape.hidden
     g = _gen(seed * 1000003 + 29 + layer * 104729, device)
     w = torch.randn(H, 3 * H, generator=g, device=device, dtype=torch.float32) * 0.02
+    return w.to(torch_dtype(spec.shape))
+
+
+def make_w_o(spec: WorkloadSpec, seed: int, layer: int = 0, device="cpu") -> torch.Tensor:
+    """W_o [H, H] row-major, N(0, 0.02^2): the output projection of a chained
+    stack's layer."""
+    H = spec.shape.hidden
+    g = _gen(seed * 1000003 + 67 + layer * 130363, device)
+    w = torch.randn(H, H, generator=g, device=device, dtype=torch.float32) * 0.02
     return w.to(torch_dtype(spec.shape))
 
 
@@ -334,13 +376,21 @@ def algorithmic_bytes_flops(spec: WorkloadSpec, meta: StepMeta, with_mass: bool 
             + out (fp32) + attn_mass (fp32);
     flops = 2*R*H*3H (projection) + 4*D*n_h*sum_r |K(r)| (QK^T and PV).
     The second key pass, padding rows and RoPE/softmax arithmetic are not
-    counted."""
+    counted. A chained stack's layer adds its output projection with the
+    residual: W_o read, x_{l+1} written in place of the fp32 out, and
+    2*R*H*H flops (the bf16 out that feeds the projection is an
+    intermediate, not counted)."""
     sh = spec.shape
     s = 2 if sh.dtype == "bf16" else 4
     H = sh.hidden
     R = meta.total_rows
-    byt = H * 3 * H * s + R * H * s + R * 2 * H * s + R * H * 4
+    byt = H * 3 * H * s + R * H * s + R * 2 * H * s
     fl = 2 * R * H * 3 * H
+    if spec.chained:
+        byt += H * H * s + R * H * s
+        fl += 2 * R * H * H
+    else:
+        byt += R * H * 4
     keys = 0
     for b in range(meta.batch):
         L = int(meta.seq_lens[b])
@@ -439,3 +489,53 @@ def make_oproj(spec: OprojSpec, seed: int, device="cpu"):
     o = torch.randn(spec.rows, spec.hidden, generator=g, device=device, dtype=torch.float32)
     w = torch.randn(spec.hidden, spec.hidden, generator=g, device=device, dtype=torch.float32) * 0.02
     return o.to(torch.bfloat16), w.to(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ toy decode loop
+@dataclasses.dataclass(frozen=True)
+class ToyConfig:
+    hidden: int = 512
+    n_heads: int = 4
+    head_dim: int = 128
+    n_layers: int = 2
+    page_size: int = 64
+    rope_theta: float = 500000.0
+    batch: int = 2
+    prompt_len: int = 64
+    gen_len: int = 64
+    window: int = 8
+    track_k: int = 8
+    tau: float = 0.5
+    seed: int = 0
+
+
+def toy_weights(cfg: ToyConfig, device="cpu"):
+    """Random bf16 weights of the toy model, from seeded generators:
+    E [V, H] ~ N(0, 1) (V = H, the last id is [MASK]); per layer Wqkv
+    [H, 3H] and W_o [H, H] ~ N(0, 0.02^2); the LM head W_lm [H, V] ~
+    N(0, 0.02^2) scaled by 8 so that some predictions are confident."""
+    H = cfg.hidden
+    g = torch.Generator(device="cpu").manual_seed(cfg.seed * 7919 + 5)
+    bf = torch.bfloat16
+    emb = torch.randn(H, H, generator=g).to(bf)
+    wqkv = [(torch.randn(H, 3 * H, generator=g) * 0.02).to(bf) for _ in range(cfg.n_layers)]
+    w_o = [(torch.randn(H, H, generator=g) * 0.02).to(bf) for _ in range(cfg.n_layers)]
+    w_lm = (torch.randn(H, H, generator=g) * 0.16).to(bf)
+    return {k: (v.to(device) if isinstance(v, torch.Tensor) else [t.to(device) for t in v])
+            for k, v in dict(emb=emb, wqkv=wqkv, w_o=w_o, w_lm=w_lm).items()}
+
+
+def toy_layout(cfg: ToyConfig):
+    """Seeded host state: prompt tokens, the [MASK]ed generation region and
+    a permuted block table. Returns (tokens [B, L] int64, block_table
+    [B, blocks] int32, num_pages)."""
+    rng = np.random.default_rng(cfg.seed)
+    B, L, ps = cfg.batch, cfg.prompt_len + cfg.gen_len, cfg.page_size
+    V = cfg.hidden
+    tokens = np.full((B, L), V - 1, np.int64)
+    tokens[:, :cfg.prompt_len] = rng.integers(0, V - 1, (B, cfg.prompt_len))
+    nblk = (L + ps - 1) // ps
+    num_pages = B * nblk + 2
+    perm = rng.permutation(num_pages).astype(np.int32)
+    bt = perm[:B * nblk].reshape(B, nblk)
+    return tokens, bt, num_pages

@@ -343,7 +343,7 @@ def verify_accept(pred, conf, draft_tokens, cu_rows, tau: float):
 # Output projection of the attention block (a "next" step after the layer)
 # --------------------------------------------------------------------------
 
-def oproj(out_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
+def oproj(out_bits: np.ndarray, w_bits: np.ndarray, residual_bits=None) -> np.ndarray:
     """The attention block's output projection y = o W_o, float64.
 
     o [R, H] holds each row's attention output with the heads side by side
@@ -353,7 +353,13 @@ def oproj(out_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
     cache write, scheduled attention) and say nothing of W_o; this is the
     plain linear map that follows attention in a transformer layer, read
     with the same conventions as Wqkv (y = x W, row-major, no bias).
+    With residual_bits (bf16 [R, H]) it returns residual + o W_o: the
+    residual stream of a transformer layer, which is how one layer's output
+    becomes the next layer's input when layers are chained.
     Returns float64 [R, H]; rounding y to bf16 is the caller's business."""
     o = bf16_bits_to_f64(out_bits)
     w = bf16_bits_to_f64(w_bits)
-    return o @ w
+    y = o @ w
+    if residual_bits is not None:
+        y = y + bf16_bits_to_f64(residual_bits)
+    return y

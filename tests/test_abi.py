@@ -80,13 +80,18 @@ def test_oproj_host_checks_without_a_gpu(lib):
     """fdllm_oproj refuses bad sizes, null and misaligned pointers before any
     CUDA call (the pointers below are never dereferenced)."""
     A, Wp, Y = 1 << 20, 2 << 20, 3 << 20          # aligned stand-in addresses
-    assert lib.fdllm_oproj(A, Wp, Y, 4, 100, None, None) == _lib.FDLLM_ERR_UNSUPPORTED
+    assert lib.fdllm_oproj(A, Wp, None, Y, 4, 100, None, None) == _lib.FDLLM_ERR_UNSUPPORTED
     assert b"multiple of 256" in lib.fdllm_last_error()
-    assert lib.fdllm_oproj(A, Wp, Y, -1, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
-    assert lib.fdllm_oproj(A, Wp, Y, 4, 0, None, None) == _lib.FDLLM_ERR_INVALID_ARG
-    assert lib.fdllm_oproj(None, Wp, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
-    assert lib.fdllm_oproj(A + 8, Wp, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    assert lib.fdllm_oproj(A, Wp, None, Y, -1, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    assert lib.fdllm_oproj(A, Wp, None, Y, 4, 0, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    assert lib.fdllm_oproj(None, Wp, None, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    assert lib.fdllm_oproj(A + 8, Wp, None, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
     assert b"16-byte aligned" in lib.fdllm_last_error()
+    assert lib.fdllm_oproj(A, Wp, A + 8, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    # y may be the residual, but must not overlap the other inputs
+    assert lib.fdllm_oproj(A, Wp, Y + 256, Y, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
+    assert b"overlaps" in lib.fdllm_last_error()
+    assert lib.fdllm_oproj(A, Wp, None, A + 256, 4, 256, None, None) == _lib.FDLLM_ERR_INVALID_ARG
     # no rows: nothing to do, nothing enqueued
-    assert lib.fdllm_oproj(None, None, None, 0, 256, None, None) == _lib.FDLLM_OK
+    assert lib.fdllm_oproj(None, None, None, None, 0, 256, None, None) == _lib.FDLLM_OK
     assert lib.fdllm_last_launch_count() == 0

@@ -121,3 +121,28 @@ def test_layer_step_bf16_out_then_oproj(name):
         y = fd.fdllm_oproj(outs[1], w_o.to(dev))
         torch.cuda.synchronize()
         _check(W.bits_np(outs[1].cpu()), W.bits_np(w_o), y.float().cpu().numpy())
+
+
+def _check_resid(o_bits, w_bits, r_bits, y_rows):
+    ref = O.oproj(o_bits, w_bits, r_bits)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    bad = np.abs(y_rows - ref) > 2.0 ** -8 * np.abs(ref) + 1e-4 * rms
+    assert not bad.any(), f"{int(bad.sum())} elements off; max err {np.abs(y_rows - ref).max():.3e}"
+
+
+@pytest.mark.parametrize("rows,hidden", [(3, 256), (130, 512), (1536, 4096)])
+def test_oproj_with_residual_and_in_place(rows, hidden):
+    """y = residual + o W_o, into a fresh buffer and in place over the
+    residual (the residual stream of a chained stack)."""
+    o, w = _case(rows, hidden, 11 + rows)
+    g = torch.Generator().manual_seed(rows)
+    r = torch.randn(rows, hidden, generator=g).to(torch.bfloat16)
+    y = fd.fdllm_oproj(o.cuda(), w.cuda(), residual=r.cuda())
+    rd = r.cuda()
+    fd.fdllm_oproj(o.cuda(), w.cuda(), y=rd, residual=rd)
+    torch.cuda.synchronize()
+    idx = np.arange(rows) if rows <= 256 else np.unique(
+        np.concatenate([[0, 127, 128, rows - 1], np.random.default_rng(1).integers(0, rows, 16)]))
+    ob, wb, rb = W.bits_np(o), W.bits_np(w), W.bits_np(r)
+    _check_resid(ob[idx], wb, rb[idx], y.float().cpu().numpy()[idx])
+    assert torch.equal(y, rd)

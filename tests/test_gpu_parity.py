@@ -13,18 +13,20 @@ from oracle import oracle as O
 from gpu_case import build_inputs, compare, run_gpu, run_oracle
 
 
-def check_dense(spec, meta, x, w, kp, vp, g):
-    """Compare a dense-x GPU run with the oracle: the plain 1e-2 * RMS bar
-    on out (1e-4 for fp32), cache values within one bf16 ulp. For bf16, a
-    step whose exact reading the bar cannot hold for (fresh v on the other
-    side of a bf16 rounding midpoint under fp32 accumulation, where that key
-    carries much of a row's attention) is held to the same bar against the
-    oracle's fp32-accumulate reading."""
+def check_dense(spec, meta, x, w, kp, vp, g, grid=False):
+    """Compare a GPU run with the oracle. bf16 grid inputs (exact fp32
+    projection) and fp32 workloads: the plain bar. bf16 continuous inputs:
+    the plain bar, or, where the oracle's own fp32-accumulate reading shows
+    it is out of reach, the bar plus twice that reading's spread."""
     o = run_oracle(spec, meta, x, w, kp, vp)
-    bf = spec.shape.dtype == "bf16"
-    compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="dense" if bf else "plain",
-            orc_f32acc=(lambda: run_oracle(spec, meta, x, w, kp, vp, accumulate="f32")) if bf
-            else None)
+    if spec.shape.dtype != "bf16":
+        compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="plain")
+    elif grid:
+        compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="grid")
+    else:
+        compare(spec, meta, g, o, W.bits_np(kp), W.bits_np(vp), mode="dense",
+                orc_f32acc=lambda: run_oracle(spec, meta, x, w, kp, vp, accumulate="f32"))
+
 
 pytestmark = pytest.mark.gpu
 
@@ -34,13 +36,36 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("seed", [0, 1])
 def test_parity_small(name, seed):
     spec = W.get_spec(name)
-    meta, x, w, kp, vp = build_inputs(spec, seed)
+    meta, x, w, kp, vp = build_inputs(spec, seed, grid=True)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    check_dense(spec, meta, x, w, kp, vp, g, grid=True)
+
+
+@pytest.mark.parametrize("name", ["small_bf16_divergent", "small_bf16_two_view"])
+def test_parity_small_continuous(name):
+    spec = W.get_spec(name)
+    meta, x, w, kp, vp = build_inputs(spec, 2)
     g = run_gpu(spec, meta, x, w, kp, vp)
     check_dense(spec, meta, x, w, kp, vp, g)
 
 
 @pytest.mark.parametrize("name", ["llada8b_b1", "b32_divergent", "two_view_b8"])
 def test_parity_full_size(name):
+    """Full size, in the launch configuration the benchmark times, on dense
+    normally shaped inputs whose projection is exact in fp32 (grid): the
+    plain 1e-2 x RMS bar."""
+    spec = W.get_spec(name)
+    meta, x, w, kp, vp = build_inputs(spec, 0, grid=True)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    check_dense(spec, meta, x, w, kp, vp, g, grid=True)
+
+
+@pytest.mark.parametrize("name", ["llada8b_b1", "b32_divergent", "two_view_b8"])
+def test_parity_full_size_continuous(name):
+    """Full size on the benchmark's own continuous inputs (x ~ N(0,1),
+    Wqkv ~ N(0, 0.02^2)): the plain bar, or, where the oracle's own
+    fp32-accumulate reading already misses it, the bar plus twice that
+    spread."""
     spec = W.get_spec(name)
     meta, x, w, kp, vp = build_inputs(spec, 0)
     g = run_gpu(spec, meta, x, w, kp, vp)
@@ -51,8 +76,9 @@ def test_parity_stacked32_sampled_layers():
     """The 32-layer stack at full size (batch 4, 8192 cached slots per
     sequence, 32 window + 64 tracked rows): every layer runs on the GPU in
     stream order through one handle over the full pools, as the benchmark
-    runs them; three sampled layers are checked against the oracle. One-hot
-    x rows make each projection exact, so the plain bound applies."""
+    runs them; three sampled layers are checked against the oracle. Dense
+    grid inputs (x ~ N(0,1) on a 1/4 grid, Wqkv ~ N(0, 0.02^2) on a 2^-10
+    grid) make each projection exact in fp32, so the plain bar applies."""
     from gpu_case import GpuResult
     spec = W.get_spec("stacked32_b4")
     sh = spec.shape
@@ -62,8 +88,8 @@ def test_parity_stacked32_sampled_layers():
     sampled = (0, 13, nl - 1)
     kp, vp = W.make_pools(spec, meta, 0, device=dev)
     pre = {l: (W.bits_np(kp[l:l + 1]), W.bits_np(vp[l:l + 1])) for l in sampled}
-    xs = [W.make_x_onehot(spec, meta, 100 + l, device=dev) for l in range(nl)]
-    ws = [W.make_w(spec, 0, layer=l, device=dev) for l in range(nl)]
+    xs = [W.make_x_grid(spec, meta, 100 + l, device=dev) for l in range(nl)]
+    ws = [W.make_w_grid(spec, 0, layer=l, device=dev) for l in range(nl)]
     ps = sh.page_size
     cache = fd.FlashCache(nl, sh.n_heads, sh.head_dim, ps, meta.num_pages, meta.max_position,
                           sh.rope_theta, sh.dtype, max_batch=meta.batch,
@@ -88,7 +114,7 @@ def test_parity_stacked32_sampled_layers():
         kb, vb = pre[l]
         o = O.layer_step(sh, kb, vb, 0, W.bits_np(xs[l]), W.bits_np(ws[l]), meta.positions,
                          meta.slots, meta.cu_rows, meta.seq_lens, meta.block_table, meta.view)
-        compare(spec, meta, g, o, kb, vb, mode="exact")
+        compare(spec, meta, g, o, kb, vb, mode="grid", label=f"stacked32_b4 layer {l}")
     cache.close()
 
 

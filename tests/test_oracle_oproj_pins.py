@@ -76,7 +76,36 @@ def pin_head_blocks() -> bool:
     return ok
 
 
-PINS = [pin_identity, pin_permutation, pin_brute_force, pin_head_blocks]
+def pin_residual_zero_weight() -> bool:
+    # W_o = 0: y is the residual row exactly
+    rng = np.random.default_rng(5)
+    r = _rand_bf16(rng, (4, 16))
+    o = _rand_bf16(rng, (4, 16))
+    y = O.oproj(o, _bits(np.zeros((16, 16))), r)
+    return bool(np.array_equal(y, O.bf16_bits_to_f64(r)))
+
+
+def pin_residual_brute_force() -> bool:
+    # residual + o W_o by a triple loop, each residual element added once
+    rng = np.random.default_rng(6)
+    R, H = 3, 8
+    o = _rand_bf16(rng, (R, H))
+    w = _rand_bf16(rng, (H, H), 0.02)
+    r = _rand_bf16(rng, (R, H))
+    ov, wv, rv = O.bf16_bits_to_f64(o), O.bf16_bits_to_f64(w), O.bf16_bits_to_f64(r)
+    y = O.oproj(o, w, r)
+    ok = True
+    for i in range(R):
+        for n in range(H):
+            acc = rv[i, n]
+            for k in range(H):
+                acc += ov[i, k] * wv[k, n]
+            ok &= abs(y[i, n] - acc) <= 1e-12 * max(1.0, abs(acc))
+    return bool(ok)
+
+
+PINS = [pin_identity, pin_permutation, pin_brute_force, pin_head_blocks, pin_residual_zero_weight,
+        pin_residual_brute_force]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -84,20 +113,36 @@ def test_oproj_pin(pin):
     assert pin()
 
 
-def _transposed(out_bits, w_bits):
-    return O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits).T
+def _with_residual(y, residual_bits):
+    return y if residual_bits is None else y + O.bf16_bits_to_f64(residual_bits)
 
 
-def _dropped_k(out_bits, w_bits):
+def _transposed(out_bits, w_bits, residual_bits=None):
+    return _with_residual(O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits).T,
+                          residual_bits)
+
+
+def _dropped_k(out_bits, w_bits, residual_bits=None):
     o, w = O.bf16_bits_to_f64(out_bits), O.bf16_bits_to_f64(w_bits)
-    return o[:, :-1] @ w[:-1, :]
+    return _with_residual(o[:, :-1] @ w[:-1, :], residual_bits)
 
 
-def _bf16_rounded(out_bits, w_bits):
-    return O.round_to_bf16(O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits))
+def _bf16_rounded(out_bits, w_bits, residual_bits=None):
+    return _with_residual(O.round_to_bf16(O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits)),
+                          residual_bits)
 
 
-@pytest.mark.parametrize("mutant", [_transposed, _dropped_k, _bf16_rounded],
+def _residual_dropped(out_bits, w_bits, residual_bits=None):
+    return O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits)
+
+
+def _residual_twice(out_bits, w_bits, residual_bits=None):
+    y = O.bf16_bits_to_f64(out_bits) @ O.bf16_bits_to_f64(w_bits)
+    return _with_residual(_with_residual(y, residual_bits), residual_bits)
+
+
+@pytest.mark.parametrize("mutant", [_transposed, _dropped_k, _bf16_rounded, _residual_dropped,
+                                    _residual_twice],
                          ids=lambda f: f.__name__)
 def test_planted_oproj_mistakes_are_caught(monkeypatch, mutant):
     monkeypatch.setattr(O, "oproj", mutant)
