@@ -828,14 +828,17 @@ def run_unfused(args):
                 ev[1].record()
         return 0
 
-    # kernels per step, counted once with the profiler (untimed)
+    # kernels per step, counted once with the torch profiler (untimed; left
+    # out under an external profiler, which the torch profiler would clash with)
     step(None)
     torch.cuda.synchronize()
-    from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        step(None)
-        torch.cuda.synchronize()
-    per_step = sum(1 for e in prof.events() if e.device_type.name == "CUDA")
+    per_step = None
+    if not args.no_launch_count:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step(None)
+            torch.cuda.synchronize()
+        per_step = sum(1 for e in prof.events() if e.device_type.name == "CUDA")
     step_ms, layer_ms, _ = time_steps(step, args.steps, args.warmup, flush)
     ms = float(np.mean(step_ms))
     roof = roofline_of(spec, meta, float(np.mean(layer_ms)) / nl / 1000.0, peaks, peak_src,
@@ -845,7 +848,7 @@ def run_unfused(args):
             "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
             "config": config_block(spec, meta, argparse.Namespace(gpus=1, seed=args.seed)),
             "layer_steps_per_s": nl / (ms / 1000.0), "roofline": roof,
-            "gpu_launches": per_step * args.steps,
+            "gpu_launches": per_step * args.steps if per_step is not None else None,
             "note": "torch/cuBLAS kernels, not this library's; selection not included"}
     if rank == 0:
         print(json.dumps(line))
@@ -1250,6 +1253,8 @@ def main(argv=None):
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the step kernel, when captured for this build")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-launch-count", action="store_true",
+                    help="unfused arm: skip counting its kernels with the torch profiler")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the table of the other layer workloads in the default run")
     args = ap.parse_args(argv)

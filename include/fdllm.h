@@ -128,9 +128,10 @@ typedef struct {
 /* Creates a handle over caller-owned pools.
  *   k_pool, v_pool: DEVICE [n_layers][num_pages][n_heads][page_size][head_dim]
  *     of cfg->dtype, 16-byte aligned. Not modified here.
- * Allocates the RoPE cos/sin tables (computed on the host in double,
- * stored fp32), the mass workspace and a device error word, and
- * synchronises `stream` once. */
+ * Allocates the RoPE cos/sin tables (computed on the host in double and
+ * kept in double: the kernels rotate q and k in double, so each rotated
+ * value is rounded to the cache dtype once), the mass workspace and a
+ * device error word, and synchronises `stream` once. */
 FDLLM_API fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, void* v_pool,
                                 void* stream, fdllm_cache** out);
 
@@ -203,10 +204,10 @@ FDLLM_API fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_
  * engine that has already given nearly all free HBM to its KV pool, or a
  * framework whose own allocator must account for every device byte.
  *   cfg, k_pool, v_pool: as for fdllm_cache_create (same rules).
- *   rope_cos, rope_sin: DEVICE fp32 [cfg->max_position][cfg->head_dim / 2],
+ *   rope_cos, rope_sin: DEVICE fp64 [cfg->max_position][cfg->head_dim / 2],
  *     16-byte aligned, owned by the caller: entry [p][i] is the cosine / sine
- *     of p * rope_theta^(-2i/head_dim), rounded to fp32 (the tables that
- *     fdllm_cache_create computes in double).
+ *     of p * rope_theta^(-2i/head_dim) in double (the tables that
+ *     fdllm_cache_create builds).
  *   layer, step, x, wqkv, positions, block_table, view_mask, out, attn_mass,
  *     stream: as for fdllm_layer_step; cfg->max_batch and
  *     cfg->max_slots_per_seq bound the step the same way.
@@ -229,7 +230,7 @@ FDLLM_API fdllm_status fdllm_select_tracked(const float* attn_mass, const int32_
  * them. No cudaMalloc, cudaFree or other device allocation happens; host
  * planning uses ordinary host memory as in fdllm_layer_step. */
 FDLLM_API fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_pool,
-                                      void* v_pool, const float* rope_cos, const float* rope_sin,
+                                      void* v_pool, const double* rope_cos, const double* rope_sin,
                                       int32_t layer, const fdllm_step* step, const void* x,
                                       const void* wqkv, const int32_t* positions,
                                       const int32_t* block_table, const int8_t* view_mask,

@@ -128,7 +128,7 @@ def fdllm_layer_step_noalloc(n_layers: int, n_heads: int, head_dim: int, page_si
     that cannot call cudaMalloc when they step (their HBM is already handed
     to a KV pool or to their own allocator). The library keeps its scratch
     in a fixed per-device array; overlapping calls on one GPU race on it.
-    rope_cos / rope_sin: caller-owned fp32 [max_position][head_dim / 2]
+    rope_cos / rope_sin: caller-owned fp64 [max_position][head_dim / 2]
     tables (see include/fdllm.h)."""
     lib = load()
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -147,7 +147,7 @@ def fdllm_layer_step_noalloc(n_layers: int, n_heads: int, head_dim: int, page_si
               _dev_ptr(slots, torch.int32, "slots"), 1 if validate else 0, _out_bf16(out))
     check_status(lib.fdllm_layer_step_noalloc(
         ctypes.byref(cfg), _dev_ptr(k_pool, tdt, "k_pool"), _dev_ptr(v_pool, tdt, "v_pool"),
-        _dev_ptr(rope_cos, torch.float32, "rope_cos"), _dev_ptr(rope_sin, torch.float32, "rope_sin"),
+        _dev_ptr(rope_cos, torch.float64, "rope_cos"), _dev_ptr(rope_sin, torch.float64, "rope_sin"),
         int(layer), ctypes.byref(st), _dev_ptr(x, None, "x"), _dev_ptr(wqkv, None, "wqkv"),
         _dev_ptr(positions, torch.int32, "positions"), _dev_ptr(block_table, torch.int32, "block_table"),
         _dev_ptr(view_mask, torch.int8, "view_mask"), _dev_ptr(out, None, "out"),

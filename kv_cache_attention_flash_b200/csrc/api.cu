@@ -334,8 +334,8 @@ struct fdllm_cache {
   void* k_pool;
   void* v_pool;
   int device;
-  float* rope_cos;
-  float* rope_sin;
+  double* rope_cos;
+  double* rope_sin;
   float* mass_part;
   size_t mass_part_floats;
   int* err;
@@ -408,21 +408,24 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
   cudaGetDevice(&h->device);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-  // RoPE tables in double on the host, stored fp32: angle p * theta^(-2i/D).
+  // RoPE tables in double: cos / sin of the angle p * theta^(-2i/D). The
+  // kernels rotate in double too, so that each rotated q / k value is
+  // rounded once, from a double close enough to the exact rotation that its
+  // bf16 (or fp32) code is the exactly rounded one.
   const int half = c.head_dim / 2;
   const size_t nt = (size_t)c.max_position * half;
-  std::vector<float> cs(nt), sn(nt);
+  std::vector<double> cs(nt), sn(nt);
   for (int p = 0; p < c.max_position; ++p)
     for (int i = 0; i < half; ++i) {
       const double inv = std::pow((double)c.rope_theta, -2.0 * i / c.head_dim);
       const double phi = (double)p * inv;
-      cs[(size_t)p * half + i] = (float)std::cos(phi);
-      sn[(size_t)p * half + i] = (float)std::sin(phi);
+      cs[(size_t)p * half + i] = std::cos(phi);
+      sn[(size_t)p * half + i] = std::sin(phi);
     }
   h->mass_part_floats = (size_t)c.n_heads * c.max_batch * c.max_slots_per_seq;
   cudaError_t e;
-  if ((e = cudaMalloc(&h->rope_cos, nt * sizeof(float))) != cudaSuccess ||
-      (e = cudaMalloc(&h->rope_sin, nt * sizeof(float))) != cudaSuccess ||
+  if ((e = cudaMalloc(&h->rope_cos, nt * sizeof(double))) != cudaSuccess ||
+      (e = cudaMalloc(&h->rope_sin, nt * sizeof(double))) != cudaSuccess ||
       (e = cudaMalloc(&h->mass_part, h->mass_part_floats * sizeof(float))) != cudaSuccess ||
       (e = cudaMalloc(&h->err, 4 * sizeof(int))) != cudaSuccess ||
       (c.dtype == FDLLM_BF16 &&
@@ -430,9 +433,9 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
     fdllm_cache_destroy(h);
     return cuda_fail(e, "cache_create: cudaMalloc");
   }
-  if ((e = cudaMemcpyAsync(h->rope_cos, cs.data(), nt * sizeof(float), cudaMemcpyHostToDevice,
+  if ((e = cudaMemcpyAsync(h->rope_cos, cs.data(), nt * sizeof(double), cudaMemcpyHostToDevice,
                            st)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(h->rope_sin, sn.data(), nt * sizeof(float), cudaMemcpyHostToDevice,
+      (e = cudaMemcpyAsync(h->rope_sin, sn.data(), nt * sizeof(double), cudaMemcpyHostToDevice,
                            st)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->err, 0, 4 * sizeof(int), st)) != cudaSuccess ||
       (h->split_flags &&
@@ -978,7 +981,7 @@ fdllm_status noalloc_scratch(cudaStream_t stream, void** addr) {
 extern "C" {
 
 fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_pool, void* v_pool,
-                                      const float* rope_cos, const float* rope_sin, int32_t layer,
+                                      const double* rope_cos, const double* rope_sin, int32_t layer,
                                       const fdllm_step* st, const void* x, const void* wqkv,
                                       const int32_t* positions, const int32_t* block_table,
                                       const int8_t* view_mask, void* out, float* attn_mass,
@@ -1046,8 +1049,8 @@ fdllm_status fdllm_layer_step_noalloc(const fdllm_cache_config* cfg, void* k_poo
       return fail(FDLLM_ERR_CUDA, "layer_step_noalloc: cuTensorMapEncodeTiled failed for the pools");
   }
   cudaGetDevice(&h.device);
-  h.rope_cos = const_cast<float*>(rope_cos);
-  h.rope_sin = const_cast<float*>(rope_sin);
+  h.rope_cos = const_cast<double*>(rope_cos);
+  h.rope_sin = const_cast<double*>(rope_sin);
   h.mass_part = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocPartOffset);
   h.mass_part_floats = kNoAllocPartFloats;
   h.err = static_cast<int*>(scratch);

@@ -66,8 +66,8 @@ struct StepArgs {
   float* mass_part;              // [n_heads][batch][row_stride] or null
   void* k_pool;
   void* v_pool;
-  const float* rope_cos;         // [max_position][head_dim/2]
-  const float* rope_sin;
+  const double* rope_cos;        // [max_position][head_dim/2]
+  const double* rope_sin;
   int* err;                      // device error word
   int hidden;
   int n_heads;

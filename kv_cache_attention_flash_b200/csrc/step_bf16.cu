@@ -107,6 +107,11 @@ struct Ctrl {
   uint64_t pv_done;
   uint64_t q_ready;       // repeated q rows written (sequences of at most 64 rows)
   uint64_t o_done;
+  uint64_t s_half;        // resident scores: the first half of the chunks' S^T is in TMEM
+  uint64_t s_all;         //   and all of them (each completes once per sequence)
+  uint64_t t_free;        // the softmax warps are done with this sequence's TMEM
+  uint64_t pv_buf[2];     // resident scores: P.V product done with P^T buffer 0 / 1
+  uint64_t p_buf[2];      //   and P^T buffer 0 / 1 written (8 softmax warps)
   uint32_t tmem_base;
   int abort;
   // per-row metadata of the group
@@ -126,8 +131,13 @@ struct Ctrl {
   int pg_phys[MAX_PAGES];   //   and their physical pages (-1: bad table entry)
   alignas(16) float lse2[BM];   // log2-sum-exp2 of the scaled scores of each row (float4 loads)
   float pm2[2][BM], pl2[2][BM];  // pass-1 partial (max, sum) per TMEM lane and warp half
+  alignas(16) float red[4][BM];  // resident scores: per-quadrant row partials
+  alignas(16) float row_m[BM];   //   row maximum (scaled, log2 domain; float4 loads)
+  alignas(16) float row_inv[BM]; //   1 / row sum of exponentials (float4 loads)
 };
 static_assert(offsetof(Ctrl, lse2) % 16 == 0, "lse2 is read as float4");
+static_assert(offsetof(Ctrl, row_m) % 16 == 0 && offsetof(Ctrl, row_inv) % 16 == 0,
+              "row_m and row_inv are read as float4");
 static_assert(sizeof(Ctrl) % 16 == 0 || true, "");
 constexpr int CTRL_OFF = PIPE_BYTES;
 constexpr int SMEM_BYTES = PIPE_BYTES + (int)sizeof(Ctrl) + 1024;
@@ -146,6 +156,10 @@ __device__ __forceinline__ bool wait_bar(Ctrl* c, uint64_t* bar, uint32_t parity
   set_err(err, kDevTimeout, site);
   atomicExch(&c->abort, 1);
   return false;
+}
+
+__device__ __forceinline__ bool aborted(Ctrl* c) {
+  return *reinterpret_cast<volatile int*>(&c->abort) != 0;
 }
 
 // 128-byte swizzled K-major operand: byte offset of the 16-byte chunk `ch`
@@ -167,20 +181,33 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void rope32(float* lo, float* hi, int pos, int c, const float* cos_t,
-                                       const float* sin_t) {
-  const float4* cp = reinterpret_cast<const float4*>(cos_t + (size_t)pos * (D / 2) + 32 * c);
-  const float4* sp = reinterpret_cast<const float4*>(sin_t + (size_t)pos * (D / 2) + 32 * c);
+// double -> float with round-to-odd: truncate toward zero, then set the
+// last bit when the value was not exact. Rounding that float to bf16 to
+// nearest even then gives the bf16 nearest to the double (Boldo and
+// Melquiond, "When double rounding is odd"), i.e. a single rounding.
+__device__ __forceinline__ float to_float_odd(double x) {
+  const float f = __double2float_rz(x);
+  const uint32_t odd = (double)f != x ? 1u : 0u;
+  return __uint_as_float(__float_as_uint(f) | odd);
+}
+
+// Rotate-half RoPE of dimensions [32c, 32c + 32) and [64 + 32c, ...) in
+// double from double cos / sin tables; the results come back as
+// round-to-odd floats for the bf16 rounding that follows.
+__device__ __forceinline__ void rope32(float* lo, float* hi, int pos, int c, const double* cos_t,
+                                       const double* sin_t) {
+  const double2* cp = reinterpret_cast<const double2*>(cos_t + (size_t)pos * (D / 2) + 32 * c);
+  const double2* sp = reinterpret_cast<const double2*>(sin_t + (size_t)pos * (D / 2) + 32 * c);
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const float4 cs = __ldg(cp + u), sn = __ldg(sp + u);
-    const float cv[4] = {cs.x, cs.y, cs.z, cs.w}, sv[4] = {sn.x, sn.y, sn.z, sn.w};
+  for (int u = 0; u < 16; ++u) {
+    const double2 cs = __ldg(cp + u), sn = __ldg(sp + u);
+    const double cv[2] = {cs.x, cs.y}, sv[2] = {sn.x, sn.y};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int t = 4 * u + e;
-      const float a = lo[t], b = hi[t];
-      lo[t] = a * cv[e] - b * sv[e];
-      hi[t] = b * cv[e] + a * sv[e];
+    for (int e = 0; e < 2; ++e) {
+      const int t = 2 * u + e;
+      const double a = lo[t], b = hi[t];
+      lo[t] = to_float_odd(fma(a, cv[e], -b * sv[e]));
+      hi[t] = to_float_odd(fma(b, cv[e], a * sv[e]));
     }
   }
 }
@@ -197,7 +224,7 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // TMEM -> registers -> RoPE -> bf16 -> q operand rows. Every lane of the
 // warp executes the TMEM loads; only valid rows are rotated and written.
 __device__ __forceinline__ void epi_q(uint32_t taddr, int qrow, bool valid, int pos,
-                                      const float* cos_t, const float* sin_t, uint8_t* q) {
+                                      const double* cos_t, const double* sin_t, uint8_t* q) {
 #pragma unroll 1
   for (int c = 0; c < 2; ++c) {
     float lo[32], hi[32];
@@ -218,7 +245,7 @@ __device__ __forceinline__ void epi_q(uint32_t taddr, int qrow, bool valid, int 
 // Pass c covers dimensions [32c, 32c + 32) and [64 + 32c, 64 + 32c + 32)
 // (the rotate-half pairs); passes [c0, c1) are done.
 __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool rotate, int pos,
-                                       const float* cos_t, const float* sin_t, uint8_t* dst,
+                                       const double* cos_t, const double* sin_t, uint8_t* dst,
                                        int c0 = 0, int c1 = 2) {
 #pragma unroll 1
   for (int c = c0; c < c1; ++c) {
@@ -257,6 +284,57 @@ __device__ __forceinline__ void lse_block(float* v, uint32_t mk, float sl2, floa
   for (int j = 0; j < NK; ++j) s4[j & 3] += ptx::ex2(fmaf(v[j], sl2, -mn));
   l = l * ptx::ex2(m - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
   m = mn;
+}
+
+// Reduction over the 32 lanes (keys) of a warp of NR row values per lane
+// (NR = 8, 16 or 32): recursive halving, so that after log2(NR) exchange
+// steps each lane holds one row, then plain butterflies over the lanes that
+// share it. Returns the reduced value of row (lane >> (5 - log2 NR)).
+template <int NR, bool kMax>
+__device__ __forceinline__ float lane_reduce_rows(float (&v)[32], int lane) {
+  constexpr int K = NR == 32 ? 5 : NR == 16 ? 4 : 3;
+  static_assert(NR == 8 || NR == 16 || NR == 32, "rows per half");
+#pragma unroll
+  for (int step = 0; step < K; ++step) {
+    const int off = 16 >> step;
+    const int n = NR >> (step + 1);   // values kept after this step
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = upper ? v[i] : v[i + n];
+      const float keep = upper ? v[i + n] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int off = (16 >> K); off >= 1; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, r, off);
+    r = kMax ? fmaxf(r, o) : r + o;
+  }
+  return r;
+}
+
+template <int NR>
+__device__ __forceinline__ void tmem_ld_rows(uint32_t taddr, float* v) {
+  if constexpr (NR == 32) ptx::tmem_ld32(taddr, v);
+  else if constexpr (NR == 16) ptx::tmem_ld16(taddr, v);
+  else ptx::tmem_ld8(taddr, v);
+}
+
+template <int NR>
+__device__ __forceinline__ void tmem_st_rows(uint32_t taddr, const float* v) {
+  if constexpr (NR == 32) ptx::tmem_st32(taddr, v);
+  else if constexpr (NR == 16) ptx::tmem_st16(taddr, v);
+  else ptx::tmem_st8(taddr, v);
+}
+
+// A sequence keeps all of its scores in TMEM (one S^T product per chunk,
+// N16 columns each, O^T later in the first chunk's columns) when its padded
+// rows are a power of two up to 64 and its chunks fit the 512 columns.
+__device__ __forceinline__ bool resident_fits(int N16, int nch) {
+  return (N16 == 16 || N16 == 32 || N16 == 64) && nch >= 1 && nch * N16 <= 512;
 }
 
 // Schedule parameter of the one-tile kernel: none.
@@ -318,6 +396,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ptx::mbar_init(&ctrl->pv_done, 1);
     ptx::mbar_init(&ctrl->q_ready, 8);
     ptx::mbar_init(&ctrl->o_done, 1);
+    ptx::mbar_init(&ctrl->s_half, 1);
+    ptx::mbar_init(&ctrl->s_all, 1);
+    ptx::mbar_init(&ctrl->t_free, 8);
+    ptx::mbar_init(&ctrl->pv_buf[0], 1);
+    ptx::mbar_init(&ctrl->pv_buf[1], 1);
+    ptx::mbar_init(&ctrl->p_buf[0], 8);
+    ptx::mbar_init(&ctrl->p_buf[1], 8);
     ctrl->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -362,7 +447,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // attention schedule counters, identical in every thread: chunk loads (K
   // or V) issued so far, S^T products, P.V products, finished sequences and
   // sequences whose q rows were repeated
-  uint32_t ring = 0, scount = 0, pcount = 0, ocount = 0, qcount = 0;
+  uint32_t ring = 0, scount = 0, ocount = 0, qcount = 0;
+  // resident scores: sequences so far (s_half / s_all completions), P.V
+  // chunks so far (P^T buffer (rp & 1), its barrier's use rp >> 1), and
+  // t_free hand-overs. Each barrier completes at most once ahead of its
+  // waiters, so its phase parity identifies the completion.
+  uint32_t rcount = 0, rpcount = 0, tcount = 0;
+  uint32_t opcount = 0;   // P.V chunks of two-pass sequences (p_full / pv_done completions)
+  int64_t last_load = -1; // producer: the last attention chunk load actually issued
   for (int ti = t_beg; ti < t_end; ++ti) {
   int g, h;
   if constexpr (kPersist) {
@@ -404,11 +496,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // x rows are read by every head's tile of the group and a head's
       // Wqkv slice by every group's tile: keep both in L2
       const uint64_t pol_keep = ptx::policy_evict_last();
+      int kissued = 0;
       for (int kb = 0; kb < nkb; ++kb) {
         const uint32_t kg = kstep0 + kb;
         const int s = kg % kStages;
         const uint32_t u = kg / kStages;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
+        if (u == 0 && aborted(ctrl)) break;
+        kissued = kb + 1;
         uint8_t* st = smem + s * kStageBytes;
         ptx::mbar_arrive_expect_tx(&ctrl->full[s], (kSplit ? B_BYTES / 3 : B_BYTES) + x_rows * BK * 2);
 #pragma unroll
@@ -429,6 +524,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         else
           ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
                                 pol_keep);
+      }
+      // after a timeout: the stages still in flight land before this CTA
+      // moves on (every earlier stage was consumed by a product that waited
+      // for it)
+      if (aborted(ctrl)) {
+        for (int kb = kissued > kStages ? kissued - kStages : 0; kb < kissued; ++kb) {
+          const uint32_t kg = kstep0 + kb;
+          ptx::mbar_wait(&ctrl->full[kg % kStages], (kg / kStages) & 1, WAIT_NS);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -718,6 +822,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // the error word holds the timeout)
   const bool gave_up = kSplit && *reinterpret_cast<volatile int*>(&ctrl->abort) != 0;
   const int nseq_g = (role == 0 && !gave_up) ? ctrl->nseq : 0;
+  auto seq_resident = [&](int q) -> bool {
+    const int n16 = (ctrl->sq_n[q] + 15) & ~15;
+    return resident_fits(n16, (ctrl->sq_npages[q] + 1) >> 1);
+  };
   for (int si = 0; si < nseq_g; ++si) {
     const int b = ctrl->sq_b[si];
     const int n = ctrl->sq_n[si];
@@ -734,6 +842,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int* xsl = ctrl->xs_slot + ctrl->sq_x0[si];
     const int* xsr = ctrl->xs_row + ctrl->sq_x0[si];
     const int nch = (npages + 1) >> 1;
+    // Resident scores (a sequence of 16, 32 or 64 padded rows whose chunks
+    // fit TMEM): one S^T = K Q^T product per chunk into its own TMEM
+    // columns, so K is read once; the softmax warps reduce the row maxima
+    // and sums across lanes and form P from the same scores; O^T
+    // accumulates in the first chunk's columns once they have been read.
+    // Otherwise the two-pass scheme below. Where this sequence or the one
+    // before it is resident, its first product waits until the softmax
+    // warps have released the earlier sequence's TMEM (t_free).
+    const bool res = resident_fits(N16, nch);
+    const bool wait_free = si > 0 && (res || seq_resident(si - 1));
+    const bool give_free = si + 1 < nseq_g && (res || seq_resident(si + 1));
     // Pass 1 keeps the rows on TMEM lanes. A sequence of at most 64 rows
     // is repeated R times (copy rho on lanes [rho*RS, rho*RS + N16)), so
     // that every lane quadrant (every SM sub-partition) holds rows; copy
@@ -750,7 +869,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // (items r0 + c); pass 2 K_0, K_1, then V_c followed by K_{c+2}, so that
     // K runs one chunk ahead of V and each load's slot was freed by a
     // product issued a chunk earlier.
-    const uint32_t r0 = ring, s0 = scount, p0 = pcount;
+    const uint32_t r0 = ring, s0 = scount;
     const int npre = nch < 2 ? nch : 2;
     const int nk2 = nch > 2 ? nch - 2 : 0;
     auto item_v2 = [&](int c) -> uint32_t {
@@ -769,7 +888,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         auto load = [&](int c, bool is_v, uint64_t pol) {
           const int s = item % NSLOT;
           const uint32_t u = item / NSLOT;
-          if (u > 0) wait_bar(ctrl, &ctrl->aempty[s], (u - 1) & 1, a.err, 10);
+          // after a timeout nothing more is issued (the slot may still be read)
+          const bool free_ok = u > 0 ? wait_bar(ctrl, &ctrl->aempty[s], (u - 1) & 1, a.err, 10)
+                                     : !aborted(ctrl);
+          if (!free_ok) {
+            ++item;
+            return;
+          }
           uint32_t bytes = 0;
           int phys[2] = {-1, -1};
           for (int pi = 0; pi < 2; ++pi) {
@@ -789,18 +914,82 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ptx::tma_load_2d_hint(dst + HALF_BYTES + pi * BOX_BYTES, map, 64, row, &ctrl->afull[s],
                                   pol);
           }
+          last_load = item;
           ++item;
         };
-        for (int c = 0; c < nch; ++c) load(c, false, pol_keep);
-        for (int c = 0; c < npre; ++c) load(c, false, pol_drop);
-        for (int c = 0; c < nch; ++c) {
-          load(c, true, pol_drop);
-          if (c + 2 < nch) load(c + 2, false, pol_drop);
+        if (res) {   // every chunk's K, then every chunk's V, each read once
+          for (int c = 0; c < nch; ++c) load(c, false, pol_drop);
+          for (int c = 0; c < nch; ++c) load(c, true, pol_drop);
+        } else {
+          for (int c = 0; c < nch; ++c) load(c, false, pol_keep);
+          for (int c = 0; c < npre; ++c) load(c, false, pol_drop);
+          for (int c = 0; c < nch; ++c) {
+            load(c, true, pol_drop);
+            if (c + 2 < nch) load(c + 2, false, pol_drop);
+          }
         }
       }
     } else if (warp == kMmaWarp) {
       // ---------------------------------------- MMA issuer
-      if (lane == 0) {
+      if (lane == 0 && wait_free) wait_bar(ctrl, &ctrl->t_free, (tcount - 1) & 1, a.err, 17);
+      if (lane == 0 && res) {
+        const uint32_t idesc_s = ptx::idesc_bf16_f32(128, N16, false, false);
+        const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, N16, true, true);
+        // S^T_c = K_c Q^T into columns [c * N16, (c + 1) * N16)
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t item = r0 + c;
+          const int s = item % NSLOT;
+          // after a timeout no product is issued
+          if (wait_bar(ctrl, &ctrl->afull[s], (item / NSLOT) & 1, a.err, 11)) {
+            ptx::tc_fence_after();
+            const uint32_t kbase = slot_base + s * SLOT_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+              const uint64_t kd = ptx::smem_desc_sw128(kbase + off, 16, 1024);
+              const uint64_t qd = ptx::smem_desc_sw128(q_base + off + qoff * 128, 16, 1024);
+              ptx::umma_f16_ss(tmem + (uint32_t)(c * N16), kd, qd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            ptx::umma_commit(&ctrl->aempty[s]);
+          }
+          if (c == (nch + 1) / 2 - 1) ptx::umma_commit(&ctrl->s_half);
+        }
+        ptx::umma_commit(&ctrl->s_all);
+        // O^T += V_c^T P_c^T into columns [0, N16) (chunk 0's scores are
+        // read before P_0 is published); P^T alternates between two buffers
+        bool any = false;
+        for (int c = 0; c < nch; ++c) {
+          const uint32_t vitem = r0 + nch + c;
+          const int vs = vitem % NSLOT;
+          const uint32_t rp = rpcount + (uint32_t)c;
+          const uint32_t pbuf = pt_base + (rp & 1u) * 32768u;
+          // per-buffer barriers: with two buffers the softmax warps can
+          // publish P_{c+1} before this thread has seen P_c, and a single
+          // barrier would then be two completions ahead of its waiter
+          if (!wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 13) ||
+              !wait_bar(ctrl, &ctrl->p_buf[rp & 1u], (rp >> 1) & 1, a.err, 14))
+            continue;   // after a timeout no product is issued
+          ptx::tc_fence_after();
+          const uint32_t vbase = slot_base + vs * SLOT_BYTES;
+          for (int pi = 0; pi < 2; ++pi) {
+            const int pidx = 2 * c + pi;
+            if (pidx >= npages || pgp[pidx] < 0) continue;
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const int ks = pi * 4 + k4;
+              const uint64_t ad = ptx::smem_desc_sw128(vbase + ks * 2048, HALF_BYTES, 1024);
+              const uint64_t bh = ptx::smem_desc_noswz(pbuf + ks * 256, 128, 2048);
+              const uint64_t bl = ptx::smem_desc_noswz(pbuf + ptl_off + ks * 256, 128, 2048);
+              ptx::umma_f16_ss(tmem, ad, bh, idesc_pv, any ? 1u : 0u);
+              ptx::umma_f16_ss(tmem, ad, bl, idesc_pv, 1u);
+              any = true;
+            }
+          }
+          ptx::umma_commit(&ctrl->aempty[vs]);
+          ptx::umma_commit(&ctrl->pv_buf[rp & 1u]);
+        }
+        ptx::umma_commit(&ctrl->o_done);
+      } else if (lane == 0) {
         const uint32_t idesc_std = ptx::idesc_bf16_f32(128, 128, false, false);
         const uint32_t idesc_s = ptx::idesc_bf16_f32(128, N16, false, false);
         const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, N16, true, true);
@@ -810,10 +999,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // on columns).
         auto issue_s = [&](uint32_t j, uint32_t item, bool transposed) {
           const int s = item % NSLOT;
-          wait_bar(ctrl, &ctrl->afull[s], (item / NSLOT) & 1, a.err, 11);
           const uint32_t idx = s0 + j;
           const uint32_t sb = idx & 1, su = idx >> 1;
-          if (su > 0) wait_bar(ctrl, &ctrl->s_empty[sb], (su - 1) & 1, a.err, 12);
+          // after a timeout no product is issued
+          if (!wait_bar(ctrl, &ctrl->afull[s], (item / NSLOT) & 1, a.err, 11)) return;
+          if (su > 0 && !wait_bar(ctrl, &ctrl->s_empty[sb], (su - 1) & 1, a.err, 12)) return;
           ptx::tc_fence_after();
           const uint32_t kbase = slot_base + s * SLOT_BYTES;
 #pragma unroll
@@ -839,8 +1029,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < nch; ++c) {
           const uint32_t vitem = item_v2(c);
           const int vs = vitem % NSLOT;
-          wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 13);
-          wait_bar(ctrl, &ctrl->p_full, (p0 + c) & 1, a.err, 14);
+          if (!wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 13) ||
+              !wait_bar(ctrl, &ctrl->p_full, (opcount + c) & 1, a.err, 14))
+            continue;   // after a timeout no product is issued
           ptx::tc_fence_after();
           const uint32_t vbase = slot_base + vs * SLOT_BYTES;
           for (int pi = 0; pi < 2; ++pi) {
@@ -919,6 +1110,152 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         return m;
       };
+
+      // ----- resident scores (see above). Thread t owns key t of every
+      // chunk; the warp pair of a lane quadrant splits the rows in halves of
+      // NR = N16 / 2 (warp half h: rows [h * NR, h * NR + NR)).
+      auto resident_softmax = [&](auto nr_const) {
+        constexpr int NR = decltype(nr_const)::value;
+        constexpr int LPR = 32 / NR;                // lanes that share a reduced row
+        const int rbase = half * NR;
+        const uint32_t cbase = tmem + tl + (uint32_t)rbase;
+        auto row_mask = [&](int c, int& slot, int& cat) -> uint32_t {
+          int xr;
+          key_info(c, slot, cat, xr);
+          const uint32_t m = vis_mask(cat, xr, rbase >> 5) >> (rbase & 31);
+          return NR == 32 ? m : (m & ((1u << NR) - 1u));
+        };
+        float acc[32];
+        // sweep 1: row maxima of the raw scores, this thread's keys (the
+        // first half of the chunks as soon as their products land), then
+        // across the lanes and the four quadrants
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = -INFINITY;
+        for (int c = 0; c < nch; ++c) {
+          int slot, cat;
+          const uint32_t mk = row_mask(c, slot, cat);
+          if (c == 0 || c == (nch + 1) / 2) {
+            wait_bar(ctrl, c == 0 ? &ctrl->s_half : &ctrl->s_all, rcount & 1, a.err, 25);
+            ptx::tc_fence_after();
+          }
+          float v[32];
+          tmem_ld_rows<NR>(cbase + (uint32_t)(c * N16), v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < NR; ++j)
+            if ((mk >> j) & 1u) acc[j] = fmaxf(acc[j], v[j]);
+        }
+        {
+          const float r = lane_reduce_rows<NR, true>(acc, lane);
+          if ((lane & (LPR - 1)) == 0) ctrl->red[quad][rbase + lane / LPR] = r;
+        }
+        named_bar(1, NSMX);
+        for (int rr = tid; rr < N16; rr += NSMX) {
+          const float m = fmaxf(fmaxf(ctrl->red[0][rr], ctrl->red[1][rr]),
+                                fmaxf(ctrl->red[2][rr], ctrl->red[3][rr]));
+          // rounding is monotone, so the scaled maximum is the maximum scaled score
+          ctrl->row_m[rr] = m * sl2;
+        }
+        named_bar(1, NSMX);
+        // sweep 2: e = 2^(s * sl2 - m) (0 where the key is not visible),
+        // summed per row, and stored back over the scores for sweep 3
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+        for (int c = 0; c < nch; ++c) {
+          int slot, cat;
+          const uint32_t mk = row_mask(c, slot, cat);
+          float v[32];
+          tmem_ld_rows<NR>(cbase + (uint32_t)(c * N16), v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j4 = 0; j4 < NR; j4 += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(ctrl->row_m + rbase + j4);
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = j4 + e;
+              v[j] = ((mk >> j) & 1u) ? ptx::ex2(fmaf(v[j], sl2, -mm[e])) : 0.f;
+              acc[j] += v[j];
+            }
+          }
+          tmem_st_rows<NR>(cbase + (uint32_t)(c * N16), v);
+        }
+        ptx::tmem_st_wait();
+        {
+          const float r = lane_reduce_rows<NR, false>(acc, lane);
+          if ((lane & (LPR - 1)) == 0) ctrl->red[quad][rbase + lane / LPR] = r;
+        }
+        named_bar(1, NSMX);
+        for (int rr = tid; rr < N16; rr += NSMX) {
+          const float l = (ctrl->red[0][rr] + ctrl->red[1][rr]) + (ctrl->red[2][rr] + ctrl->red[3][rr]);
+          ctrl->row_inv[rr] = l > 0.f ? 1.f / l : 0.f;
+        }
+        named_bar(1, NSMX);
+        // sweep 3, chunk by chunk: P = e / l, the per-key mass, P^T (bf16 hi
+        // + lo) for the P.V product, in two buffers that alternate
+        for (int c = 0; c < nch; ++c) {
+          int slot, cat;
+          (void)row_mask(c, slot, cat);
+          const int pidx = 2 * c + (t >> 6);
+          const bool loaded = pidx < npages && pgp[pidx] >= 0;
+          const uint32_t rp = rpcount + (uint32_t)c;
+          uint8_t* pth = smem + PT_OFF + (rp & 1u) * 32768u;
+          uint8_t* ptl = pth + ptl_off;
+          float v[32];
+          tmem_ld_rows<NR>(cbase + (uint32_t)(c * N16), v);
+          ptx::tmem_ld_wait();
+          uint32_t ph[NR / 2], pq[NR / 2];
+          float msum = 0.f;
+#pragma unroll
+          for (int j4 = 0; j4 < NR; j4 += 4) {
+            const float4 i4 = *reinterpret_cast<const float4*>(ctrl->row_inv + rbase + j4);
+            const float ii[4] = {i4.x, i4.y, i4.z, i4.w};
+            float pv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pv[e] = v[j4 + e] * ii[e];
+            msum += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+            ptx::split_bf16(pv[0], pv[1], ph[j4 >> 1], pq[j4 >> 1]);
+            ptx::split_bf16(pv[2], pv[3], ph[(j4 >> 1) + 1], pq[(j4 >> 1) + 1]);
+          }
+          // this chunk's scores are read (chunk 0's columns take O^T next)
+          ptx::tc_fence_before();
+          // both halves add into the zeroed mass row: two addends, so the
+          // result does not depend on their order
+          if (part && cat != 0) atomicAdd(part + slot, msum);
+          const uint32_t vitem = r0 + nch + c;
+          const int vs = vitem % NSLOT;
+          if (loaded && cat == 0) {
+            // V rows of keys nobody attends may hold anything: zero them
+            wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 22);
+            uint8_t* vrow = smem + SLOT_OFF + vs * SLOT_BYTES + half * HALF_BYTES +
+                            (t >> 6) * BOX_BYTES + (t & 63) * 128;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
+          }
+          // this P^T buffer is free once the product two chunks back completed
+          if (rp >= 2) wait_bar(ctrl, &ctrl->pv_buf[rp & 1u], ((rp >> 1) - 1) & 1, a.err, 23);
+#pragma unroll
+          for (int g8 = 0; g8 < NR / 8; ++g8) {
+            const int nb = (rbase >> 3) + g8;      // 8-row block of the sequence
+            *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) =
+                make_uint4(ph[4 * g8], ph[4 * g8 + 1], ph[4 * g8 + 2], ph[4 * g8 + 3]);
+            *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) =
+                make_uint4(pq[4 * g8], pq[4 * g8 + 1], pq[4 * g8 + 2], pq[4 * g8 + 3]);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&ctrl->p_buf[rp & 1u]);
+        }
+      };
+      if (res) {
+        if (N16 == 16)
+          resident_softmax(std::integral_constant<int, 8>{});
+        else if (N16 == 32)
+          resident_softmax(std::integral_constant<int, 16>{});
+        else
+          resident_softmax(std::integral_constant<int, 32>{});
+      } else {
 
       // ----- repeated q rows for pass 1 (sequences of at most 64 rows):
       // lane t holds row t % RS. A 128-byte row's swizzle phase depends on
@@ -1084,8 +1421,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
         }
-        // The P^T buffers are free once the previous P.V product completed.
-        const uint32_t pidx_g = p0 + c;
+        // The P^T buffers are free once the previous P.V product completed
+        // (pv_done counts the two-pass chunks only). Earlier resident chunks
+        // used the buffers too; their products completed before this
+        // sequence began (o_done of that sequence).
+        const uint32_t pidx_g = opcount + c;
         if (pidx_g > 0) wait_bar(ctrl, &ctrl->pv_done, (pidx_g - 1) & 1, a.err, 23);
         uint8_t* pth = smem + PT_OFF;
         uint8_t* ptl = pth + ptl_off;
@@ -1107,14 +1447,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctrl->p_full);
       }
+      }   // two-pass scheme
       // ----- O^T -> out (thread t = head dimension t; the halves split rows)
+      const int nsub_o = N16 >> 4;
+      const uint32_t o_col = res ? 0u : TM_O;
       wait_bar(ctrl, &ctrl->o_done, ocount & 1, a.err, 24);
       ptx::tc_fence_after();
       if (!a.out_bf16) {
         float* o32 = static_cast<float*>(a.out);
-        for (int k = half; k < nsub; k += 2) {
+        for (int k = half; k < nsub_o; k += 2) {
           float v[16];
-          ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
+          ptx::tmem_ld16(tmem + tl + o_col + 16 * k, v);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -1124,9 +1467,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       } else {
         __nv_bfloat16* o16 = static_cast<__nv_bfloat16*>(a.out);
-        for (int k = half; k < nsub; k += 2) {
+        for (int k = half; k < nsub_o; k += 2) {
           float v[16];
-          ptx::tmem_ld16(tmem + tl + TM_O + 16 * k, v);
+          ptx::tmem_ld16(tmem + tl + o_col + 16 * k, v);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -1137,12 +1480,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       ptx::tc_fence_before();
+      // this sequence's TMEM is free for the next sequence's products
+      __syncwarp();
+      if (give_free && lane == 0) ptx::mbar_arrive(&ctrl->t_free);
     }
-    ring = r0 + 3 * nch;
-    scount = s0 + 2 * nch;
-    pcount = p0 + nch;
+    ring = r0 + (res ? 2 : 3) * nch;
+    scount = s0 + (res ? 0 : 2 * nch);
     ++ocount;
-    if (!wide) ++qcount;
+    if (!wide && !res) ++qcount;
+    if (res) {
+      ++rcount;
+      rpcount += nch;
+    } else {
+      opcount += nch;
+    }
+    if (give_free) ++tcount;
   }
 
   // ================================================================ tile end
@@ -1155,8 +1507,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ptx::mbar_wait(&ctrl->mma_done, 1, WAIT_NS);
   }
   if (warp == kProducerWarp && lane == 0 && ring > 0) {
+    // only loads that were issued (none after a timeout)
     for (uint32_t it = ring > NSLOT ? ring - NSLOT : 0; it < ring; ++it)
-      ptx::mbar_wait(&ctrl->afull[it % NSLOT], (it / NSLOT) & 1, WAIT_NS);
+      if ((int64_t)it <= last_load)
+        ptx::mbar_wait(&ctrl->afull[it % NSLOT], (it / NSLOT) & 1, WAIT_NS);
   }
   __syncwarp();
   if constexpr (kPersist) {

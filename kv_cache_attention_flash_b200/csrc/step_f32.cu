@@ -118,18 +118,19 @@ __global__ void __launch_bounds__(NT)
       const int lr = rb + r;
       const bool ok = rpage[lr] >= 0;
       const int pos = ok ? rpos[lr] : 0;
-      const float cs = a.rope_cos[(size_t)pos * half + i];
-      const float sn = a.rope_sin[(size_t)pos * half + i];
+      // rotation in double from the double tables, rounded to fp32 once
+      const double cs = a.rope_cos[(size_t)pos * half + i];
+      const double sn = a.rope_sin[(size_t)pos * half + i];
       const float* tr = tmp + r * C3;
-      const float q1 = tr[i], q2 = tr[i + half];
-      const float k1 = tr[D + i], k2 = tr[D + i + half];
-      qs[lr * D + i] = ok ? q1 * cs - q2 * sn : 0.f;
-      qs[lr * D + i + half] = ok ? q2 * cs + q1 * sn : 0.f;
+      const double q1 = tr[i], q2 = tr[i + half];
+      const double k1 = tr[D + i], k2 = tr[D + i + half];
+      qs[lr * D + i] = ok ? (float)fma(q1, cs, -q2 * sn) : 0.f;
+      qs[lr * D + i + half] = ok ? (float)fma(q2, cs, q1 * sn) : 0.f;
       if (ok) {
         const size_t off = layer_base + ((size_t)rpage[lr] * a.n_heads + h) * ps * D +
                            (size_t)(rslot[lr] % ps) * D;
-        kpool[off + i] = k1 * cs - k2 * sn;
-        kpool[off + i + half] = k2 * cs + k1 * sn;
+        kpool[off + i] = (float)fma(k1, cs, -k2 * sn);
+        kpool[off + i + half] = (float)fma(k2, cs, k1 * sn);
         vpool[off + i] = tr[2 * D + i];
         vpool[off + i + half] = tr[2 * D + i + half];
       }

@@ -32,12 +32,11 @@ SCRATCH_FLOATS = ((8 << 20) - 256) // 4
 
 
 def rope_tables(max_position, head_dim, theta, device):
-    """cos / sin of p * theta^(-2i/head_dim) in float64, stored fp32."""
+    """cos / sin of p * theta^(-2i/head_dim), float64 (the caller's tables)."""
     half = head_dim // 2
     inv = np.power(np.float64(np.float32(theta)), -2.0 * np.arange(half) / head_dim)
     phi = np.arange(max_position, dtype=np.float64)[:, None] * inv[None, :]
-    return (torch.from_numpy(np.cos(phi).astype(np.float32)).to(device),
-            torch.from_numpy(np.sin(phi).astype(np.float32)).to(device))
+    return (torch.from_numpy(np.cos(phi)).to(device), torch.from_numpy(np.sin(phi)).to(device))
 
 
 def bf16_ulp(v):
