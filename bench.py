@@ -17,8 +17,11 @@ LLaDA-8B layer shape, bf16).
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
 events on the launching stream with an L2 flush (a 256 MB write) between
-steps, outside the events; barrier + synchronize on both sides; the total is
-the max over ranks. Under torchrun each rank runs its own batch (independent
+steps, outside the events, followed by a short device-side spin so that the
+host has queued the step before its start event is reached (the events time
+GPU work; the end-to-end figure keeps host planning and copies in its timed
+region); barrier + synchronize on both sides; the total is the max over
+ranks. Under torchrun each rank runs its own batch (independent
 sequences: weak scaling, no collective on the data path).
 
 One JSON line is printed by rank 0.
@@ -282,9 +285,9 @@ class UnfusedStep:
     the probabilities. Same inputs, pool layout and results (within the
     parity bar) as the fused step; it exists only to measure what the fusion
     saves. The projection and the scores take bf16 operands with fp32
-    results (cuBLAS), so q and k are rounded once, after RoPE, as in the
-    fused step; P V runs in fp32 with TF32 allowed, which is exact for the
-    bf16-valued v and rounds P to 11 bits.
+    results (cuBLAS); RoPE runs in double and rounds q and k to bf16 once,
+    as in the fused step; P V runs in fp32 with TF32 allowed, which is exact
+    for the bf16-valued v and rounds P to 11 bits.
 
     The padded shapes and the row / key index tensors depend only on cu_rows
     and seq_lens (host metadata, as in the fused path) and are built once;
@@ -298,8 +301,8 @@ class UnfusedStep:
         half = D // 2
         inv = np.float64(np.float32(sh.rope_theta)) ** (-2.0 * np.arange(half) / D)
         phi = np.arange(meta.max_position, dtype=np.float64)[:, None] * inv[None, :]
-        self.cos = torch.from_numpy(np.cos(phi).astype(np.float32)).to(device)
-        self.sin = torch.from_numpy(np.sin(phi).astype(np.float32)).to(device)
+        self.cos = torch.from_numpy(np.cos(phi)).to(device)
+        self.sin = torch.from_numpy(np.sin(phi)).to(device)
         B = meta.batch
         cu = meta.cu_rows
         n = np.diff(cu)
@@ -325,10 +328,23 @@ class UnfusedStep:
         self.scale = 1.0 / float(np.sqrt(D))
 
     def _rope(self, u, c, s):
+        """Rotate-half RoPE in double from double tables, returned as bf16
+        rounded once: double -> float with round-to-odd (truncate toward
+        zero, set the last bit when inexact), then float -> bf16 to nearest
+        even, which together round the double to the nearest bf16 (Boldo and
+        Melquiond, "When double rounding is odd")."""
         half = self.sh.head_dim // 2
-        u = u.float()
+        u = u.double()
         a, b = u[..., :half], u[..., half:]
-        return torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+        d = torch.cat([a * c - b * s, b * c + a * s], dim=-1)
+        f = d.float()
+        away = f.double().abs() > d.abs()
+        fb = f.view(torch.int32)
+        fb = torch.where(away, fb - 1, fb)                 # toward zero
+        f = fb.view(torch.float32)
+        inexact = f.double() != d
+        f = torch.where(inexact, (f.view(torch.int32) | 1).view(torch.float32), f)
+        return f.to(torch.bfloat16)
 
     def step(self, layer, k_pool, v_pool, x, w, pos, slots, view, bt, out, mass):
         sh, meta = self.sh, self.meta
@@ -345,8 +361,8 @@ class UnfusedStep:
         p = pos.long()
         c = self.cos[p][:, None, :]
         s = self.sin[p][:, None, :]
-        qr = self._rope(q, c, s).to(bf)
-        kr = self._rope(k, c, s).to(bf)
+        qr = self._rope(q, c, s)
+        kr = self._rope(k, c, s)
         # 3. cache write through the block table (index_put_)
         sl = slots.long()
         btl = bt.long()
@@ -642,6 +658,17 @@ def roofline_of(spec, meta, kern_s, peaks, peak_src, kernel_name, traffic=None):
             "roofline_us": max(t_hbm, t_tc) * 1e6, "frac_of_roofline": max(t_hbm, t_tc) / kern_s}
 
 
+def hold_device(us: float = 1000.0):
+    """Keeps the stream busy for about `us` microseconds (a device-side spin,
+    outside the timed region) so that the host has queued the whole step
+    before the start event is reached: the events then time the GPU work,
+    not host planning and launch latency. The end-to-end figure keeps the
+    host in its timed region."""
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is not None:
+        sleep(int(us * 2000))      # cycles at about 2 GHz
+
+
 def time_steps(step_fn, steps, warmup, flush, ev_layers=True):
     """Runs `warmup` untimed steps, then `steps` steps bracketed by CUDA
     events on the current stream with an L2 flush between them (outside the
@@ -659,6 +686,7 @@ def time_steps(step_fn, steps, warmup, flush, ev_layers=True):
     launches = 0
     for i in range(steps):
         flush.fill_(i & 0xFF)
+        hold_device()
         ev_s[i].record()
         launches += step_fn((ev_ls[i], ev_le[i]) if ev_layers else None)
         ev_e[i].record()
@@ -956,6 +984,7 @@ def run_verify(args):
     t_wall0 = time.time()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
+        hold_device()
         ev_s[i].record()
         launches += step()
         ev_e[i].record()
@@ -1115,6 +1144,7 @@ def run_oproj(args):
     t_wall0 = time.time()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
+        hold_device()
         ev_s[i].record()
         launches += step()
         ev_e[i].record()

