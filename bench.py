@@ -147,7 +147,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -175,7 +175,7 @@ class ClockSampler:
     def summary(self):
         rows = []
         for t, line in self.samples:
-            if self.window and not (self.window[0] - 0.05 <= t <= self.window[1] + 0.05):
+            if self.window and not (self.window[0] - 0.1 <= t <= self.window[1] + 0.1):
                 continue
             p = [x.strip() for x in line.split(",")]
             if len(p) < 9:

@@ -660,10 +660,13 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
     }
     plan.group_seq0[groups.size()] = k;
     plan.n_groups = (int)groups.size();
-    // Modelled duration of a group's tile on B200 (us, fitted to measured
-    // tile timelines): the projection grows with the number of x boxes (one
-    // per power-of-two piece of each sequence's padded rows), attention
-    // with the 128-key chunks, a little more for wider sequences.
+    // Modelled duration of a group's tile on B200 (us, least-squares fits
+    // to measured per-tile timelines): the projection grows with the number
+    // of x boxes (one per power-of-two piece of each sequence's padded
+    // rows), attention with the 128-key chunks, a little more for wider
+    // sequences. Sequences whose scores stay resident in TMEM (16, 32 or 64
+    // padded rows whose context chunks fit 512 columns) pay more per
+    // sequence and less per chunk than the two-pass ones.
     for (const Grp& gp : groups) {
       int nbox = 0;
       double attn = 0.0;
@@ -671,9 +674,13 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
         nbox += __builtin_popcount((unsigned)(n16(b) / 16));
         const int ctx = (st->seq_lens[b] + c.page_size - 1) / c.page_size;
         const int extra = (rows_of(b) + c.page_size - 1) / c.page_size + 1;
-        attn += 0.53 + ((ctx + extra + 1) / 2) * (2.58 + 0.144 * (n16(b) / 16));
+        const int chunks = (ctx + extra + 1) / 2;
+        const int w = n16(b);
+        const bool resident = (w == 16 || w == 32 || w == 64) && ((ctx + 1) / 2) * w <= 512;
+        attn += resident ? 1.58 + chunks * (1.61 + 0.319 * (w / 16))
+                         : 0.53 + chunks * (2.58 + 0.144 * (w / 16));
       }
-      gcost.push_back(46.9 + 2.93 * nbox + attn);
+      gcost.push_back(59.2 + 2.0 * nbox + attn);
     }
   }
   const int ng = plan.n_groups;

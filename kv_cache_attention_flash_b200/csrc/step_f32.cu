@@ -195,10 +195,20 @@ __global__ void __launch_bounds__(NT)
           if (vis)
             off = layer_base + ((size_t)page * a.n_heads + h) * ps * D + (size_t)(slot % ps) * D;
         }
+        // q . k over D (a multiple of 32): 16-byte loads of the key row,
+        // several in flight (keys of the 32 lanes are different rows)
         float s = 0.f;
         if (vis) {
-          for (int d = 0; d < D; ++d) s = fmaf(qs[r * D + d], kp[off + d], s);
-          s *= scale;
+          const float4* k4 = reinterpret_cast<const float4*>(kp + off);
+          const float4* q4 = reinterpret_cast<const float4*>(qs + r * D);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+          for (int d4 = 0; d4 < D / 4; ++d4) {
+            const float4 kv = __ldg(k4 + d4);
+            const float4 qv = q4[d4];
+            s4[d4 & 3] = fmaf(qv.x, kv.x, fmaf(qv.y, kv.y, fmaf(qv.z, kv.z, fmaf(qv.w, kv.w, s4[d4 & 3]))));
+          }
+          s = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * scale;
         }
         if (pass == 0) {
           if (vis) {
@@ -211,11 +221,15 @@ __global__ void __launch_bounds__(NT)
           }
         } else {
           const float p = vis ? expf(s - lse) : 0.f;
+#pragma unroll 4
           for (int t = 0; t < 32; ++t) {
             const float pt = __shfl_sync(0xffffffffu, p, t);
             const size_t offt = __shfl_sync(0xffffffffu, off, t);
-            if (pt != 0.f)
-              for (int u = 0; u < D / 32; ++u) o[u] = fmaf(pt, vp[offt + u * 32 + lane], o[u]);
+            if (pt != 0.f) {
+#pragma unroll
+              for (int u = 0; u < MAXD / 32; ++u)
+                if (u < D / 32) o[u] = fmaf(pt, __ldg(vp + offt + u * 32 + lane), o[u]);
+            }
           }
           if (part) {
             pbuf[warp][lane] = p;
