@@ -66,7 +66,15 @@ def load_peaks():
 # (dram__bytes_read.sum + dram__bytes_write.sum), with the code hashes of the
 # sources it was captured on: the kernel, its PTX helpers and the host code
 # that plans its launch. The figure is reported only while all three match.
-CAPTURED_TRAFFIC = {}
+CAPTURED_TRAFFIC = {
+    "b32_divergent": {
+        "bytes": 783267072.0,     # 724.95 MB read + 58.32 MB written, one launch
+        "sources": ["74dc2982d14adbcae91472b3f5ed01e311929a173c789f70c1e5573ed147451b",
+                    "be391d302227a2ef2fe5128f6ea54d3e927a312868f880e0d405437ecf91a423",
+                    "f8854e1e241ad568d316e6e6ccbd4e206f5d57ddd64b5c73740d61d765e7ef10"],
+        "source": "ncu --set full, one launch (profiles/step_bf16_b32_divergent.md)",
+    },
+}
 
 
 def captured_traffic(name: str):
@@ -347,6 +355,11 @@ class UnfusedStep:
         return f.to(torch.bfloat16)
 
     def step(self, layer, k_pool, v_pool, x, w, pos, slots, view, bt, out, mass):
+        torch.cuda.nvtx.range_push("unfused_layer_step")
+        self._step(layer, k_pool, v_pool, x, w, pos, slots, view, bt, out, mass)
+        torch.cuda.nvtx.range_pop()
+
+    def _step(self, layer, k_pool, v_pool, x, w, pos, slots, view, bt, out, mass):
         sh, meta = self.sh, self.meta
         H, nh, D, ps = sh.hidden, sh.n_heads, sh.head_dim, sh.page_size
         R, B = meta.total_rows, meta.batch
