@@ -36,7 +36,10 @@
 //   wastes no MMA rows: S^T = K Q^T (keys on lanes, the sequence's rows on
 //   columns) gives the exact probabilities, whose per-key sums over the
 //   rows are the attention mass (one thread per key, no cross-thread
-//   reduction), and O^T += V^T P^T takes P^T as bf16 hi + lo parts. The
+//   reduction), and O^T += V^T P^T takes P^T as bf16 hi + lo parts, the lo
+//   rows stacked after the hi rows so that one product of twice the width
+//   accumulates both (O^T hi and lo in adjacent column ranges, summed when
+//   out is stored). The
 //   Flash-Verify two-view rule (paragraph 3 of the same page) decides
 //   visibility of fresh view keys.
 #include <cuda.h>
@@ -331,7 +334,8 @@ __device__ __forceinline__ void tmem_st_rows(uint32_t taddr, const float* v) {
 }
 
 // A sequence keeps all of its scores in TMEM (one S^T product per chunk,
-// N16 columns each, O^T later in the first chunk's columns) when its padded
+// N16 columns each, O^T hi and lo later in the first two chunks' columns,
+// or the unused columns after a single chunk) when its padded
 // rows are a power of two up to 64 and its chunks fit the 512 columns.
 __device__ __forceinline__ bool resident_fits(int N16, int nch) {
   return (N16 == 16 || N16 == 32 || N16 == 64) && nch >= 1 && nch * N16 <= 512;
@@ -845,8 +849,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Resident scores (a sequence of 16, 32 or 64 padded rows whose chunks
     // fit TMEM): one S^T = K Q^T product per chunk into its own TMEM
     // columns, so K is read once; the softmax warps reduce the row maxima
-    // and sums across lanes and form P from the same scores; O^T
-    // accumulates in the first chunk's columns once they have been read.
+    // and sums across lanes and form P from the same scores; O^T hi and lo
+    // accumulate in the first two chunks' columns once both have been read.
     // Otherwise the two-pass scheme below. Where this sequence or the one
     // before it is resident, its first product waits until the softmax
     // warps have released the earlier sequence's TMEM (t_free).
@@ -862,7 +866,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int R = N16 <= 32 ? 4 : (N16 <= 64 ? 2 : 1);
     const int RS = 128 / R;
     const int KR = 128 / R;
-    const uint32_t ptl_off = wide ? 32768u : 16384u;   // P^T lo after hi
+    const uint32_t ptl_off = (uint32_t)N16 * 256u;   // P^T lo rows right after the hi rows
     float* part = a.mass_part ? a.mass_part + ((size_t)h * plan.batch + b) * plan.row_stride
                               : nullptr;
     // Chunk loads of this sequence, in ring order: pass 1 K_0 .. K_{nch-1}
@@ -934,7 +938,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0 && wait_free) wait_bar(ctrl, &ctrl->t_free, (tcount - 1) & 1, a.err, 17);
       if (lane == 0 && res) {
         const uint32_t idesc_s = ptx::idesc_bf16_f32(128, N16, false, false);
-        const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, N16, true, true);
+        const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 2 * N16, true, true);
         // S^T_c = K_c Q^T into columns [c * N16, (c + 1) * N16)
         for (int c = 0; c < nch; ++c) {
           const uint32_t item = r0 + c;
@@ -955,8 +959,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (c == (nch + 1) / 2 - 1) ptx::umma_commit(&ctrl->s_half);
         }
         ptx::umma_commit(&ctrl->s_all);
-        // O^T += V_c^T P_c^T into columns [0, N16) (chunk 0's scores are
-        // read before P_0 is published); P^T alternates between two buffers
+        // O^T += V_c^T P_c^T into columns [0, 2 N16): hi rows of P^T into
+        // [0, N16), lo rows into [N16, 2 N16). Chunks 0 and 1 own those
+        // columns, so the first product also waits for P_1 (its scores read).
+        // P^T alternates between two buffers.
         bool any = false;
         for (int c = 0; c < nch; ++c) {
           const uint32_t vitem = r0 + nch + c;
@@ -969,6 +975,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!wait_bar(ctrl, &ctrl->afull[vs], (vitem / NSLOT) & 1, a.err, 13) ||
               !wait_bar(ctrl, &ctrl->p_buf[rp & 1u], (rp >> 1) & 1, a.err, 14))
             continue;   // after a timeout no product is issued
+          if (c == 0 && nch > 1 &&
+              !wait_bar(ctrl, &ctrl->p_buf[(rp + 1) & 1u], ((rp + 1) >> 1) & 1, a.err, 14))
+            continue;
           ptx::tc_fence_after();
           const uint32_t vbase = slot_base + vs * SLOT_BYTES;
           for (int pi = 0; pi < 2; ++pi) {
@@ -978,10 +987,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int k4 = 0; k4 < 4; ++k4) {
               const int ks = pi * 4 + k4;
               const uint64_t ad = ptx::smem_desc_sw128(vbase + ks * 2048, HALF_BYTES, 1024);
-              const uint64_t bh = ptx::smem_desc_noswz(pbuf + ks * 256, 128, 2048);
-              const uint64_t bl = ptx::smem_desc_noswz(pbuf + ptl_off + ks * 256, 128, 2048);
-              ptx::umma_f16_ss(tmem, ad, bh, idesc_pv, any ? 1u : 0u);
-              ptx::umma_f16_ss(tmem, ad, bl, idesc_pv, 1u);
+              const uint64_t bd = ptx::smem_desc_noswz(pbuf + ks * 256, 128, 2048);
+              ptx::umma_f16_ss(tmem, ad, bd, idesc_pv, any ? 1u : 0u);
               any = true;
             }
           }
@@ -992,7 +999,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       } else if (lane == 0) {
         const uint32_t idesc_std = ptx::idesc_bf16_f32(128, 128, false, false);
         const uint32_t idesc_s = ptx::idesc_bf16_f32(128, N16, false, false);
-        const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, N16, true, true);
+        const uint32_t idesc_pv = ptx::idesc_bf16_f32(128, 2 * N16, true, true);
         // Score product number j of this sequence from chunk-load `item`:
         // pass 1 S = Q K^T (rows of the whole group on lanes, keys on
         // columns), pass 2 S^T = K Q^T (keys on lanes, this sequence's rows
@@ -1046,10 +1053,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const uint64_t ad = ptx::smem_desc_sw128(vbase + ks * 2048, HALF_BYTES, 1024);
               // B = P^T: N-major core matrices without swizzle: 8-key
               // groups 128 B apart (LBO), 8-row blocks 2048 B apart (SBO).
-              const uint64_t bh = ptx::smem_desc_noswz(pt_base + ks * 256, 128, 2048);
-              const uint64_t bl = ptx::smem_desc_noswz(pt_base + ptl_off + ks * 256, 128, 2048);
-              ptx::umma_f16_ss(tmem + TM_O, ad, bh, idesc_pv, any ? 1u : 0u);
-              ptx::umma_f16_ss(tmem + TM_O, ad, bl, idesc_pv, 1u);
+              const uint64_t bd = ptx::smem_desc_noswz(pt_base + ks * 256, 128, 2048);
+              ptx::umma_f16_ss(tmem + TM_O, ad, bd, idesc_pv, any ? 1u : 0u);
               any = true;
             }
           }
@@ -1204,21 +1209,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float v[32];
           tmem_ld_rows<NR>(cbase + (uint32_t)(c * N16), v);
           ptx::tmem_ld_wait();
-          uint32_t ph[NR / 2], pq[NR / 2];
+          // this chunk's scores are read (chunks 0 and 1 take O^T next)
+          ptx::tc_fence_before();
+          // this P^T buffer is free once the product two chunks back
+          // completed; P^T is then written eight rows at a time
+          if (rp >= 2) wait_bar(ctrl, &ctrl->pv_buf[rp & 1u], ((rp >> 1) - 1) & 1, a.err, 23);
           float msum = 0.f;
 #pragma unroll
-          for (int j4 = 0; j4 < NR; j4 += 4) {
-            const float4 i4 = *reinterpret_cast<const float4*>(ctrl->row_inv + rbase + j4);
-            const float ii[4] = {i4.x, i4.y, i4.z, i4.w};
-            float pv[4];
+          for (int g8 = 0; g8 < NR / 8; ++g8) {
+            uint32_t ph[4], pq[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) pv[e] = v[j4 + e] * ii[e];
-            msum += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-            ptx::split_bf16(pv[0], pv[1], ph[j4 >> 1], pq[j4 >> 1]);
-            ptx::split_bf16(pv[2], pv[3], ph[(j4 >> 1) + 1], pq[(j4 >> 1) + 1]);
+            for (int j4 = 0; j4 < 8; j4 += 4) {
+              const int j = 8 * g8 + j4;
+              const float4 i4 = *reinterpret_cast<const float4*>(ctrl->row_inv + rbase + j);
+              const float p0 = v[j] * i4.x, p1 = v[j + 1] * i4.y;
+              const float p2 = v[j + 2] * i4.z, p3 = v[j + 3] * i4.w;
+              msum += (p0 + p1) + (p2 + p3);
+              ptx::split_bf16(p0, p1, ph[j4 >> 1], pq[j4 >> 1]);
+              ptx::split_bf16(p2, p3, ph[(j4 >> 1) + 1], pq[(j4 >> 1) + 1]);
+            }
+            const int nb = (rbase >> 3) + g8;      // 8-row block of the sequence
+            *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+            *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
           }
-          // this chunk's scores are read (chunk 0's columns take O^T next)
-          ptx::tc_fence_before();
           // both halves add into the zeroed mass row: two addends, so the
           // result does not depend on their order
           if (part && cat != 0) atomicAdd(part + slot, msum);
@@ -1232,16 +1245,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
-          }
-          // this P^T buffer is free once the product two chunks back completed
-          if (rp >= 2) wait_bar(ctrl, &ctrl->pv_buf[rp & 1u], ((rp >> 1) - 1) & 1, a.err, 23);
-#pragma unroll
-          for (int g8 = 0; g8 < NR / 8; ++g8) {
-            const int nb = (rbase >> 3) + g8;      // 8-row block of the sequence
-            *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) =
-                make_uint4(ph[4 * g8], ph[4 * g8 + 1], ph[4 * g8 + 2], ph[4 * g8 + 3]);
-            *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) =
-                make_uint4(pq[4 * g8], pq[4 * g8 + 1], pq[4 * g8 + 2], pq[4 * g8 + 3]);
           }
           fence_async_smem();
           __syncwarp();
@@ -1373,7 +1376,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 21);
         ptx::tc_fence_after();
         const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0);
-        uint32_t ph[4][8], pq[4][8];
+        // The P^T buffer is free once the previous P.V product completed
+        // (pv_done counts the two-pass chunks only; earlier resident chunks'
+        // products completed before this sequence began, at that sequence's
+        // o_done). P^T is then written eight rows at a time.
+        const uint32_t pidx_g = opcount + c;
+        if (pidx_g > 0) wait_bar(ctrl, &ctrl->pv_done, (pidx_g - 1) & 1, a.err, 23);
+        uint8_t* pth = smem + PT_OFF;
+        uint8_t* ptl = pth + ptl_off;
         float mass2[2] = {0.f, 0.f};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -1385,20 +1395,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float4* l4 = reinterpret_cast<const float4*>(ctrl->lse2 + 16 * k);
             ptx::tmem_ld_wait();
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              const float4 ll = l4[j4];
-              const int j = 4 * j4;
-              const float e0 = ptx::ex2(fmaf(v[j], sl2, -ll.x));
-              const float e1 = ptx::ex2(fmaf(v[j + 1], sl2, -ll.y));
-              const float e2 = ptx::ex2(fmaf(v[j + 2], sl2, -ll.z));
-              const float e3 = ptx::ex2(fmaf(v[j + 3], sl2, -ll.w));
-              const float q0 = ((m16 >> j) & 1u) ? e0 : 0.f;
-              const float q1 = ((m16 >> (j + 1)) & 1u) ? e1 : 0.f;
-              const float q2 = ((m16 >> (j + 2)) & 1u) ? e2 : 0.f;
-              const float q3 = ((m16 >> (j + 3)) & 1u) ? e3 : 0.f;
-              mass2[j4 & 1] += (q0 + q1) + (q2 + q3);
-              ptx::split_bf16(q0, q1, ph[u][j >> 1], pq[u][j >> 1]);
-              ptx::split_bf16(q2, q3, ph[u][(j >> 1) + 1], pq[u][(j >> 1) + 1]);
+            for (int g8 = 0; g8 < 2; ++g8) {
+              uint32_t ph[4], pq[4];
+#pragma unroll
+              for (int jj = 0; jj < 2; ++jj) {
+                const int j4 = 2 * g8 + jj;
+                const float4 ll = l4[j4];
+                const int j = 4 * j4;
+                const float e0 = ptx::ex2(fmaf(v[j], sl2, -ll.x));
+                const float e1 = ptx::ex2(fmaf(v[j + 1], sl2, -ll.y));
+                const float e2 = ptx::ex2(fmaf(v[j + 2], sl2, -ll.z));
+                const float e3 = ptx::ex2(fmaf(v[j + 3], sl2, -ll.w));
+                const float q0 = ((m16 >> j) & 1u) ? e0 : 0.f;
+                const float q1 = ((m16 >> (j + 1)) & 1u) ? e1 : 0.f;
+                const float q2 = ((m16 >> (j + 2)) & 1u) ? e2 : 0.f;
+                const float q3 = ((m16 >> (j + 3)) & 1u) ? e3 : 0.f;
+                mass2[j4 & 1] += (q0 + q1) + (q2 + q3);
+                ptx::split_bf16(q0, q1, ph[2 * jj], pq[2 * jj]);
+                ptx::split_bf16(q2, q3, ph[2 * jj + 1], pq[2 * jj + 1]);
+              }
+              const int nb = 2 * k + g8;     // 8-row block of the sequence
+              *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+              *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
             }
           }
         }
@@ -1421,34 +1439,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = z;
         }
-        // The P^T buffers are free once the previous P.V product completed
-        // (pv_done counts the two-pass chunks only). Earlier resident chunks
-        // used the buffers too; their products completed before this
-        // sequence began (o_done of that sequence).
-        const uint32_t pidx_g = opcount + c;
-        if (pidx_g > 0) wait_bar(ctrl, &ctrl->pv_done, (pidx_g - 1) & 1, a.err, 23);
-        uint8_t* pth = smem + PT_OFF;
-        uint8_t* ptl = pth + ptl_off;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int k = 2 * u + half;
-          if (k < nsub) {
-#pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-              const int nb = 2 * k + g8;     // 8-row block of the sequence
-              *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) =
-                  make_uint4(ph[u][4 * g8], ph[u][4 * g8 + 1], ph[u][4 * g8 + 2], ph[u][4 * g8 + 3]);
-              *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) =
-                  make_uint4(pq[u][4 * g8], pq[u][4 * g8 + 1], pq[u][4 * g8 + 2], pq[u][4 * g8 + 3]);
-            }
-          }
-        }
         fence_async_smem();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&ctrl->p_full);
       }
       }   // two-pass scheme
-      // ----- O^T -> out (thread t = head dimension t; the halves split rows)
+      // ----- O^T -> out (thread t = head dimension t; the halves split
+      // rows): the sum of the hi and lo column ranges
       const int nsub_o = N16 >> 4;
       const uint32_t o_col = res ? 0u : TM_O;
       wait_bar(ctrl, &ctrl->o_done, ocount & 1, a.err, 24);
@@ -1458,7 +1455,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int k = half; k < nsub_o; k += 2) {
           float v[16];
           ptx::tmem_ld16(tmem + tl + o_col + 16 * k, v);
+          float w2[16];
+          ptx::tmem_ld16(tmem + tl + o_col + (uint32_t)N16 + 16 * k, w2);
           ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] += w2[j];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int rr = 16 * k + j;
@@ -1470,7 +1471,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int k = half; k < nsub_o; k += 2) {
           float v[16];
           ptx::tmem_ld16(tmem + tl + o_col + 16 * k, v);
+          float w2[16];
+          ptx::tmem_ld16(tmem + tl + o_col + (uint32_t)N16 + 16 * k, w2);
           ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] += w2[j];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int rr = 16 * k + j;
