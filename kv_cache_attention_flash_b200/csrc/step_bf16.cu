@@ -266,6 +266,51 @@ __device__ __forceinline__ void epi_kv(uint32_t taddr, int row, bool valid, bool
   }
 }
 
+// q and k of dimensions [32c, 32c + 32) and their rotate-half partners
+// [64 + 32c, ...) of this lane's row, in two sub-passes of 16 pairs: each
+// cos / sin value is loaded once for both q and k. The rotation is the one
+// of rope32 (double, round-to-odd), so the results are the same bits.
+__device__ __forceinline__ void epi_qk(uint32_t trow, int c, int qrow, int row, bool valid, int pos,
+                                       const double* cos_t, const double* sin_t, uint8_t* q,
+                                       uint8_t* kst) {
+#pragma unroll 1
+  for (int s = 0; s < 2; ++s) {
+    const int d0 = 32 * c + 16 * s;            // first (lo) dimension of the sub-pass
+    float qlo[16], qhi[16], klo[16], khi[16];
+    ptx::tmem_ld16(trow + d0, qlo);
+    ptx::tmem_ld16(trow + 64 + d0, qhi);
+    ptx::tmem_ld16(trow + 128 + d0, klo);
+    ptx::tmem_ld16(trow + 192 + d0, khi);
+    ptx::tmem_ld_wait();
+    if (!valid) continue;
+    const double2* cp = reinterpret_cast<const double2*>(cos_t + (size_t)pos * (D / 2) + d0);
+    const double2* sp = reinterpret_cast<const double2*>(sin_t + (size_t)pos * (D / 2) + d0);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const double2 cs = __ldg(cp + u), sn = __ldg(sp + u);
+      const double cv[2] = {cs.x, cs.y}, sv[2] = {sn.x, sn.y};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = 2 * u + e;
+        const double a = qlo[t], b = qhi[t];
+        qlo[t] = to_float_odd(fma(a, cv[e], -b * sv[e]));
+        qhi[t] = to_float_odd(fma(b, cv[e], a * sv[e]));
+        const double ka = klo[t], kb = khi[t];
+        klo[t] = to_float_odd(fma(ka, cv[e], -kb * sv[e]));
+        khi[t] = to_float_odd(fma(kb, cv[e], ka * sv[e]));
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int ch = d0 / 8 + u;               // 16-byte chunk of the d-half
+      *reinterpret_cast<uint4*>(q + sw128(qrow, ch)) = pack8(qlo + 8 * u);
+      *reinterpret_cast<uint4*>(q + HALF_BYTES + sw128(qrow, ch)) = pack8(qhi + 8 * u);
+      *reinterpret_cast<uint4*>(kst + swz256(row, ch)) = pack8(klo + 8 * u);
+      *reinterpret_cast<uint4*>(kst + swz256(row, 8 + ch)) = pack8(khi + 8 * u);
+    }
+  }
+}
+
 // Running log2-domain max m and sum l of one row over NK more scores v
 // (raw S values; the scale sl2 = log2(e)/sqrt(D) is applied in the
 // exponent's FMA). Keys whose bit in mk is clear are dropped before
@@ -753,12 +798,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       else if (role == 2)
         epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF,
                warp < 4 ? 0 : 1, warp < 4 ? 1 : 2);
-    } else if (warp < 4) {
-      epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
-      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, 0, 1);
     } else {
-      epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF);
-      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, 1, 2);
+      // warp half c: q and k of dimensions [32c, 32c + 32) (+ partners),
+      // then the v pass c
+      const int c = warp >> 2;
+      epi_qk(trow, c, ctrl->row_q[i], i, valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF,
+             smem + KST_OFF);
+      epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, c, c + 1);
     }
   }
   ptx::tc_fence_before();
