@@ -54,6 +54,18 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
+PROBE_SRC = os.path.join(CSRC, "mma_rate.cu")
+PROBE = os.path.join(PKG, "mma_rate")
+
+
+def build_probe() -> str:
+    """Builds the tcgen05.mma issue-rate measurement program (a standalone
+    executable beside the library; not used by the library)."""
+    subprocess.check_call([nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
+                           "-std=c++17", "-I", CSRC, "-o", PROBE, PROBE_SRC, "-lcuda"])
+    return PROBE
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
