@@ -164,19 +164,19 @@ FDLLM_API void fdllm_cache_destroy(fdllm_cache* cache);
  * Writes: out, attn_mass, and for every row the k/v of every head into its
  * slot; no other cache byte changes. Within one step no sequence may read a
  * slot another sequence writes.
- * A handle's device workspace (mass partials, error word, the flags of
- * steps whose tiles are split over three CTAs) serves one step at a time:
- * steps on one handle must not run concurrently (issue them on one stream,
- * or order the streams).
- * Steps with few tiles (three CTAs per tile fit on the SMs at once, e.g. a
- * single sequence) split each tile over three CTAs, and the attending CTA
- * waits, bounded to one second, for flags that the two cache-writing CTAs
- * set. If other work on the same GPU (kernels on other streams or in other
- * processes, a green context) keeps those CTAs off the SMs for that long,
- * the wait gives up: that tile's out and attn_mass are then wrong and the
- * step records FDLLM_ERR_TIMEOUT in the device error word. With
- * step->validate = 0 the call itself still returns FDLLM_OK, so callers
- * that share the GPU must call fdllm_check to see it. */
+ * A handle's device workspace (mass partials, error word) serves one step
+ * at a time: steps on one handle must not run concurrently (issue them on
+ * one stream, or order the streams).
+ * Steps with few tiles (four CTAs per tile fit on the SMs, e.g. a single
+ * sequence; hidden a multiple of 256) run each tile as a cluster of four
+ * CTAs that split the projection's K range and exchange partial sums
+ * through distributed shared memory; the attending CTA waits, bounded to
+ * one second, for the two CTAs that write the tile's k and v rows to the
+ * cache. The four CTAs of a cluster are scheduled together, so the wait
+ * only runs out if that work stalls: the tile's out and attn_mass are then
+ * wrong and the step records FDLLM_ERR_TIMEOUT in the device error word.
+ * With step->validate = 0 the call itself still returns FDLLM_OK, so
+ * callers must call fdllm_check to see it. */
 FDLLM_API fdllm_status fdllm_layer_step(fdllm_cache* cache, int32_t layer, const fdllm_step* step,
                               const void* x, const void* wqkv, const int32_t* positions,
                               const int32_t* block_table, const int8_t* view_mask, void* out,
@@ -323,9 +323,9 @@ FDLLM_API fdllm_status fdllm_check(fdllm_cache* cache, void* stream);
  * counterpart). Faults are made on the host; nothing here traps, faults or
  * hangs the GPU.
  *   FDLLM_INJECT_SPLIT_FLAG_TIMEOUT: in the next fdllm_layer_step on `cache`
- *     that splits its tiles over three CTAs, the attending CTAs wait for a
- *     flag value the cache-writing CTAs never store, bounded to `wait_ns`
- *     nanoseconds (1 .. 1e9) instead of one second. When the wait runs out
+ *     that runs its tiles as four-CTA clusters, the k / v writing CTAs
+ *     withhold their signal to the attending CTA, whose wait is bounded to
+ *     `wait_ns` nanoseconds (1 .. 1e9) instead of one second. When it runs out
  *     the CTA records FDLLM_ERR_TIMEOUT in the device error word and skips
  *     its attention, issuing no further load or product; that step's out
  *     rows are left unwritten and its attention mass is zero. The next

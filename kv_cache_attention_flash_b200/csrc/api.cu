@@ -32,8 +32,8 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-// Bound of the split tiles' cross-CTA flag wait (the other in-kernel waits
-// use the same one second).
+// Bound of a split tile's wait for its k / v owners (the other in-kernel
+// waits use the same one second).
 constexpr uint64_t kFlagWaitNs = 1000000000ull;
 
 thread_local std::string g_last_error;
@@ -339,8 +339,8 @@ struct fdllm_cache {
   float* mass_part;
   size_t mass_part_floats;
   int* err;
-  uint32_t* split_flags;   // [kSplitMaxTiles][k, v] for three-CTA tiles (bf16 only)
-  uint32_t split_epoch;    // value the flags of the latest such launch are set to
+  uint32_t split_epoch;    // counts cluster split-K launches (failure injection sets the
+                           // kernel's wait epoch apart from it)
   int32_t inject_kind;     // pending failure injection (fdllm_inject_fault), 0 = none
   int64_t inject_wait_ns;
 };
@@ -427,9 +427,7 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
   if ((e = cudaMalloc(&h->rope_cos, nt * sizeof(double))) != cudaSuccess ||
       (e = cudaMalloc(&h->rope_sin, nt * sizeof(double))) != cudaSuccess ||
       (e = cudaMalloc(&h->mass_part, h->mass_part_floats * sizeof(float))) != cudaSuccess ||
-      (e = cudaMalloc(&h->err, 4 * sizeof(int))) != cudaSuccess ||
-      (c.dtype == FDLLM_BF16 &&
-       (e = cudaMalloc(&h->split_flags, 2 * kSplitMaxTiles * sizeof(uint32_t))) != cudaSuccess)) {
+      (e = cudaMalloc(&h->err, 4 * sizeof(int))) != cudaSuccess) {
     fdllm_cache_destroy(h);
     return cuda_fail(e, "cache_create: cudaMalloc");
   }
@@ -438,9 +436,6 @@ fdllm_status fdllm_cache_create(const fdllm_cache_config* cfg, void* k_pool, voi
       (e = cudaMemcpyAsync(h->rope_sin, sn.data(), nt * sizeof(double), cudaMemcpyHostToDevice,
                            st)) != cudaSuccess ||
       (e = cudaMemsetAsync(h->err, 0, 4 * sizeof(int), st)) != cudaSuccess ||
-      (h->split_flags &&
-       (e = cudaMemsetAsync(h->split_flags, 0, 2 * kSplitMaxTiles * sizeof(uint32_t), st)) !=
-           cudaSuccess) ||
       (e = cudaStreamSynchronize(st)) != cudaSuccess) {
     fdllm_cache_destroy(h);
     return cuda_fail(e, "cache_create: upload");
@@ -455,7 +450,6 @@ void fdllm_cache_destroy(fdllm_cache* h) {
   cudaFree(h->rope_sin);
   cudaFree(h->mass_part);
   cudaFree(h->err);
-  cudaFree(h->split_flags);
   delete h;
 }
 
@@ -706,7 +700,6 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
   a.num_pages = c.num_pages;
   a.max_position = c.max_position;
   a.out_bf16 = st->out_bf16;
-  a.split_flags = nullptr;
   a.split_epoch = 0;
   a.split_wait_epoch = 0;
   a.flag_wait_ns = kFlagWaitNs;
@@ -725,31 +718,23 @@ fdllm_status fdllm_layer_step(fdllm_cache* h, int32_t layer, const fdllm_step* s
       if (!encode_wqkv_5d(&tw, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim, 3))
         return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv)");
       const TileSched& ts = tile_schedule(gcost, c.n_heads);
-      // Few tiles: three CTAs per tile (q + attention, k, v), so that three
-      // times as many SMs stream the weights, when all of them fit at once.
+      // Few tiles: a cluster of four CTAs per tile splits the projection's
+      // K range, so that four times as many SMs stream the weights and
+      // issue the products.
       const int tiles = ng * c.n_heads;
-      const int sms = sm_count();
-      CUtensorMap tw1;
-      const void* tw1p = nullptr;
-      a.split_flags = nullptr;
-      a.split_epoch = 0;
-      if (ts.n_bins == 0 && h->split_flags && sms > 0 && 3 * tiles <= sms &&
-          tiles <= kSplitMaxTiles) {
-        if (!encode_wqkv_5d(&tw1, wqkv, (uint64_t)H, (uint64_t)c.n_heads, (uint64_t)c.head_dim, 1))
-          return fail(FDLLM_ERR_CUDA, "layer_step: cuTensorMapEncodeTiled failed (wqkv block)");
-        tw1p = &tw1;
-        if (++h->split_epoch == 0) h->split_epoch = 1;   // flags start at 0
-        a.split_flags = h->split_flags;
+      const bool split = ts.n_bins == 0 && step_bf16_split_ok(tiles, H, sm_count());
+      if (split) {
+        ++h->split_epoch;
         a.split_epoch = h->split_epoch;
         a.split_wait_epoch = h->split_epoch;
         if (h->inject_kind == FDLLM_INJECT_SPLIT_FLAG_TIMEOUT) {
-          // a value no writer stores this launch: the attending CTAs' waits run out
+          // the k / v owners withhold their arrivals: rank 0's wait runs out
           a.split_wait_epoch = h->split_epoch ^ 0x80000000u;
           a.flag_wait_ns = (uint64_t)h->inject_wait_ns;
           h->inject_kind = 0;
         }
       }
-      e = launch_step_bf16(plan, ts, a, txp, &tw, tw1p, &h->tmap_k, &h->tmap_v, s);
+      e = launch_step_bf16(plan, ts, a, txp, &tw, &h->tmap_k, &h->tmap_v, split, s);
     } else {
       e = launch_step_f32(plan, a, s);
     }

@@ -45,7 +45,6 @@ struct StepPlan {
 // n_bins == 0 the one-tile kernel runs instead, CTA i on tile i (group-major
 // order). The schedule travels as a kernel parameter, so it is kept small
 // (a larger parameter block costs launch time).
-constexpr int kSplitMaxTiles = 256;   // tiles of a three-CTA-per-tile launch
 constexpr int kMaxSchedTiles = 1024;
 constexpr int kMaxSchedBins = 160;
 struct TileSched {
@@ -76,12 +75,11 @@ struct StepArgs {
   int num_pages;
   int max_position;
   int out_bf16;
-  // three CTAs per tile (few tiles): per tile two flags [k, v], set to
-  // split_epoch when that block is in the cache; null = one CTA per tile
-  uint32_t* split_flags;
+  // cluster split-K tiles (few tiles): the k / v owners arrive on rank 0's
+  // kv_ready barrier only when split_wait_epoch == split_epoch (a test sets
+  // them apart to withhold the arrivals), and rank 0 waits at most
+  // flag_wait_ns nanoseconds for them
   uint32_t split_epoch;
-  // value the attending CTA of a split tile waits for (split_epoch, except
-  // under failure injection) and the bound of that wait in nanoseconds
   uint32_t split_wait_epoch;
   uint64_t flag_wait_ns;
 };
@@ -94,12 +92,14 @@ struct StepArgs {
 cudaError_t launch_oproj(const void* tmap_o, const void* tmap_w, int bn, const void* residual,
                          void* y, int rows, int hidden, int32_t* status, cudaStream_t stream);
 size_t oproj_smem_bytes();
-// tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows.
-// tmap_w1: the one-block view of Wqkv (box {64, 64, 2, 1, 1}), used when
-// a.split_flags is set.
+// tmap_x: x tensor maps with boxes of 16, 32, 64 and 128 rows. split: one
+// cluster of 4 CTAs per tile (the K range of the projection split four
+// ways); only where step_bf16_split_ok(tiles, hidden, SM count) holds and
+// the schedule is empty.
 cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
-                             const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
-                             const void* tmap_k, const void* tmap_v, cudaStream_t stream);
+                             const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                             const void* tmap_v, bool split, cudaStream_t stream);
+bool step_bf16_split_ok(int tiles, int hidden, int sms);
 cudaError_t launch_step_f32(const StepPlan& plan, const StepArgs& a, cudaStream_t stream);
 cudaError_t launch_mass_reduce(const StepPlan& plan, const float* part, float* mass, int n_heads,
                                cudaStream_t stream);

@@ -65,9 +65,13 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES; // 64 KB
 constexpr int PIPE_BYTES = STAGES * STAGE_BYTES;
 // A split tile's CTA loads one of the q, k, v blocks (a third of B): its
 // 32 KB stages make a ring twice as deep in the same bytes.
-constexpr int SPLIT_STAGE_BYTES = A_BYTES + B_BYTES / 3;
-constexpr int SPLIT_STAGES = PIPE_BYTES / SPLIT_STAGE_BYTES;   // 6
-static_assert(SPLIT_STAGES * SPLIT_STAGE_BYTES == PIPE_BYTES, "split ring");
+// Cluster split-K (few tiles): each of the 4 CTAs of a tile's cluster
+// accumulates q | k | v over a quarter of the K range; the partials meet in
+// the owners' shared memory (q: rank 0, k: rank 1, v: rank 2), one fp32
+// [32 column quads][128 rows][4] slot of 64 KB per sending rank.
+constexpr int CL_RANKS = 4;
+constexpr int CL_SLOT_BYTES = 65536;
+static_assert(3 * CL_SLOT_BYTES <= PIPE_BYTES, "cluster partial slots");
 constexpr int TMEM_COLS = 512;
 constexpr int NTHREADS = 320;        // warps 0-7: epilogue / softmax (two per TMEM quadrant),
                                       // warp 8: TMA producer, warp 9: MMA issuer and TMEM owner
@@ -99,8 +103,8 @@ constexpr int QREP_OFF = PT_OFF + 32768;
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
 
 struct Ctrl {
-  uint64_t full[SPLIT_STAGES];    // STAGES used, or SPLIT_STAGES in a split tile
-  uint64_t empty[SPLIT_STAGES];
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
   uint64_t mma_done;
   uint64_t afull[NSLOT];
   uint64_t aempty[NSLOT];
@@ -115,6 +119,7 @@ struct Ctrl {
   uint64_t t_free;        // the softmax warps are done with this sequence's TMEM
   uint64_t pv_buf[2];     // resident scores: P.V product done with P^T buffer 0 / 1
   uint64_t p_buf[2];      //   and P^T buffer 0 / 1 written (8 softmax warps)
+  uint64_t kv_ready;      // cluster split-K, rank 0: the k and v owners' rows are in the cache
   uint32_t tmem_base;
   int abort;
   // per-row metadata of the group
@@ -227,9 +232,10 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
 // TMEM -> registers -> RoPE -> bf16 -> q operand rows. Every lane of the
 // warp executes the TMEM loads; only valid rows are rotated and written.
 __device__ __forceinline__ void epi_q(uint32_t taddr, int qrow, bool valid, int pos,
-                                      const double* cos_t, const double* sin_t, uint8_t* q) {
+                                      const double* cos_t, const double* sin_t, uint8_t* q,
+                                      int c0 = 0, int c1 = 2) {
 #pragma unroll 1
-  for (int c = 0; c < 2; ++c) {
+  for (int c = c0; c < c1; ++c) {
     float lo[32], hi[32];
     ptx::tmem_ld32(taddr + 32 * c, lo);
     ptx::tmem_ld32(taddr + 64 + 32 * c, hi);
@@ -393,13 +399,18 @@ struct NoSched {
 
 // kPersist: a persistent CTA runs the tiles of its schedule bin; otherwise
 // CTA i runs tile i.
-// kSplit (few tiles): three CTAs per tile. CTAs 2t and 2t+1 project tile
-// t's k and v blocks only and write them to the cache, then publish them
-// through a flag (release); CTA 2T + t projects q, keeps it on chip, waits
-// for both flags (acquire, bounded) and runs the attention. Each CTA then
-// streams a third of the head's Wqkv slice. The writers come first in block
-// order and never wait, so the readers' waits end even when not every CTA
-// is resident at once.
+// kSplit (few tiles): a cluster of 4 CTAs per tile splits the projection's
+// K range in four (each CTA streams a quarter of the head's Wqkv slice and
+// issues a quarter of the products). After a cluster barrier every rank
+// sends the fp32 partials of the blocks it does not own to their owners'
+// shared memory (q: rank 0, k: rank 1, v: rank 2); after a second barrier
+// each owner adds them to its own partial in TMEM, in rank order. The k and
+// v owners write their rows to the cache and arrive on rank 0's kv_ready
+// barrier; rank 0 keeps q on chip, waits for kv_ready (bounded) and runs
+// the attention. Both cluster barriers are reached by every thread of every
+// rank on every path (all other waits are bounded), and no CTA reads or
+// writes another's shared memory after the second one except for those
+// two arrivals on rank 0, which waits for them before it goes on.
 template <bool kPersist, bool kSplit>
 __global__ void __launch_bounds__(NTHREADS, 1)
     step_bf16_kernel(const __grid_constant__ StepPlan plan,
@@ -410,7 +421,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      const __grid_constant__ CUtensorMap tmap_x64,
                      const __grid_constant__ CUtensorMap tmap_x128,
                      const __grid_constant__ CUtensorMap tmap_w,
-                     const __grid_constant__ CUtensorMap tmap_w1,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v) {
   extern __shared__ uint8_t smem_raw[];
@@ -423,12 +433,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int lane = tid & 31;
   const int H = a.hidden;
   const int nkb = H / BK;
-  constexpr int kStages = kSplit ? SPLIT_STAGES : STAGES;
-  constexpr int kStageBytes = kSplit ? SPLIT_STAGE_BYTES : STAGE_BYTES;
+  constexpr int kStages = STAGES;
+  constexpr int kStageBytes = STAGE_BYTES;
   const int layer = plan.layer;
 
   if (tid == 0) {
-    for (int s = 0; s < (kSplit ? SPLIT_STAGES : STAGES); ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&ctrl->full[s], 1);
       ptx::mbar_init(&ctrl->empty[s], 1);
     }
@@ -452,6 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ptx::mbar_init(&ctrl->pv_buf[1], 1);
     ptx::mbar_init(&ctrl->p_buf[0], 8);
     ptx::mbar_init(&ctrl->p_buf[1], 8);
+    ptx::mbar_init(&ctrl->kv_ready, 2);
     ctrl->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -476,17 +487,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // Tiles of this CTA (a persistent CTA runs several, one after another;
   // barrier phases, schedule counters and TMEM carry over between them).
   int t_beg = 0, t_end = 1;
-  // role: 0 = q and attention (everything when not split), 1 = k, 2 = v
+  // role (the rank in a split tile's cluster): 0 = q and attention
+  // (everything when not split), 1 = k, 2 = v, 3 = a partial only; the
+  // rank's quarter of the projection K steps is [kb0, kb1)
   int role = 0;
   int tile_id = (int)blockIdx.x;
+  int kb0 = 0, kb1 = nkb;
   if constexpr (kSplit) {
-    const int T = (int)gridDim.x / 3;
-    if ((int)blockIdx.x < 2 * T) {
-      role = 1 + ((int)blockIdx.x & 1);
-      tile_id = (int)blockIdx.x >> 1;
-    } else {
-      tile_id = (int)blockIdx.x - 2 * T;
-    }
+    role = (int)ptx::cluster_ctarank();
+    tile_id = (int)blockIdx.x / CL_RANKS;
+    kb0 = role * (nkb / CL_RANKS);
+    kb1 = kb0 + nkb / CL_RANKS;
   }
   if constexpr (kPersist) {
     t_beg = sched.bin0[blockIdx.x];
@@ -545,16 +556,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // x rows are read by every head's tile of the group and a head's
       // Wqkv slice by every group's tile: keep both in L2
       const uint64_t pol_keep = ptx::policy_evict_last();
-      int kissued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const uint32_t kg = kstep0 + kb;
+      int kissued = kb0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t kg = kstep0 + (kb - kb0);
         const int s = kg % kStages;
         const uint32_t u = kg / kStages;
         if (u > 0 && !wait_bar(ctrl, &ctrl->empty[s], (u - 1) & 1, a.err, 1)) break;
         if (u == 0 && aborted(ctrl)) break;
         kissued = kb + 1;
         uint8_t* st = smem + s * kStageBytes;
-        ptx::mbar_arrive_expect_tx(&ctrl->full[s], (kSplit ? B_BYTES / 3 : B_BYTES) + x_rows * BK * 2);
+        ptx::mbar_arrive_expect_tx(&ctrl->full[s], B_BYTES + x_rows * BK * 2);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           if (i < nbox) {
@@ -567,19 +578,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // this head's q, k and v column blocks of Wqkv, two 64-column halves
         // each: one 48 KB box of the 5-D view (column, K row, half, block,
         // head), laid out as six [64 K rows][64 columns] sub-boxes
-        if constexpr (kSplit)   // this CTA's block only (q, k or v): two sub-boxes
-          ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w1, 0, kb * BK, 0, role, h, &ctrl->full[s],
-                                pol_keep);
-        else
-          ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
-                                pol_keep);
+        ptx::tma_load_5d_hint(st + A_BYTES, &tmap_w, 0, kb * BK, 0, 0, h, &ctrl->full[s],
+                              pol_keep);
       }
       // after a timeout: the stages still in flight land before this CTA
       // moves on (every earlier stage was consumed by a product that waited
       // for it)
       if (aborted(ctrl)) {
-        for (int kb = kissued > kStages ? kissued - kStages : 0; kb < kissued; ++kb) {
-          const uint32_t kg = kstep0 + kb;
+        for (int kb = kissued - kStages > kb0 ? kissued - kStages : kb0; kb < kissued; ++kb) {
+          const uint32_t kg = kstep0 + (kb - kb0);
           ptx::mbar_wait(&ctrl->full[kg % kStages], (kg / kStages) & 1, WAIT_NS);
         }
       }
@@ -588,8 +595,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {   // MMA issuer
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, 128, false, true);
       constexpr uint32_t idesc256 = ptx::idesc_bf16_f32(BM, 256, false, true);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const uint32_t kg = kstep0 + kb;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t kg = kstep0 + (kb - kb0);
         const int s = kg % kStages;
         const uint32_t u = kg / kStages;
         if (!wait_bar(ctrl, &ctrl->full[s], u & 1, a.err, 2)) break;
@@ -604,17 +611,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // K groups 1024 bytes apart; K16 slice = 16 rows = 2 KB. q and k
           // (four boxes, 256 columns) go in one N=256 product, which reads
           // the A tile from shared memory once for both; v is N=128.
-          if constexpr (kSplit) {
-            // the one block, into its columns of the fused layout
-            const uint64_t b1 = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
-            ptx::umma_f16_ss(tmem + 128 * role, ad, b1, idesc, (kb | kk) != 0 ? 1u : 0u);
-          } else {
-            const uint64_t bqk = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
-            ptx::umma_f16_ss(tmem, ad, bqk, idesc256, (kb | kk) != 0 ? 1u : 0u);
-            const uint64_t bv = ptx::smem_desc_sw128(b_base + 4 * BOX_BYTES + kk * 2048,
-                                                     BOX_BYTES, 1024);
-            ptx::umma_f16_ss(tmem + 256, ad, bv, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
+          const uint32_t acc = (kb != kb0 || kk != 0) ? 1u : 0u;
+          const uint64_t bqk = ptx::smem_desc_sw128(b_base + kk * 2048, BOX_BYTES, 1024);
+          ptx::umma_f16_ss(tmem, ad, bqk, idesc256, acc);
+          const uint64_t bv = ptx::smem_desc_sw128(b_base + 4 * BOX_BYTES + kk * 2048,
+                                                   BOX_BYTES, 1024);
+          ptx::umma_f16_ss(tmem + 256, ad, bv, idesc, acc);
         }
         ptx::umma_commit(&ctrl->empty[s]);
       }
@@ -780,6 +782,81 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const bool acc_ok = wait_bar(ctrl, &ctrl->mma_done, 0, a.err, 3);
   __syncwarp();
   ptx::tc_fence_after();
+  if constexpr (kSplit) {
+    // Every rank's partial is final and every rank's ring is idle, so the
+    // partial slots (in the ring region) may be written. Each rank sends
+    // the blocks it does not own; thread (quadrant, half) moves the 64
+    // columns `half` of its row. Only the lane quadrants that hold the
+    // group's rows travel.
+    int lanes_used = 0;
+    for (int q = seq_a; q < seq_b; ++q) {
+      const int b = plan.seq_order[q];
+      const int top = plan.seq_qoff[b] + ((plan.cu_rows[b + 1] - plan.cu_rows[b] + 15) & ~15);
+      lanes_used = top > lanes_used ? top : lanes_used;
+    }
+    const int quads_used = (lanes_used + 31) >> 5;
+    ptx::tc_fence_before();
+    ptx::cluster_sync();
+    ptx::tc_fence_after();
+    if (warp < 8 && (warp & 3) < quads_used) {
+      const int quad = warp & 3, hh = warp >> 2;
+      const int row = quad * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+      const uint32_t sbase = ptx::smem_u32(smem);
+      for (int b = 0; b < 3; ++b) {
+        if (b == role) continue;
+        const int slot = role < b ? role : role - 1;
+        const uint32_t rbase = ptx::mapa_shared(sbase + (uint32_t)(slot * CL_SLOT_BYTES), (uint32_t)b);
+#pragma unroll 1
+        for (int j = 0; j < 2; ++j) {
+          float v[32];
+          ptx::tmem_ld32(trow + 128 * b + 64 * hh + 32 * j, v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const int c4 = 16 * hh + 8 * j + i4;   // column quad of the block
+            ptx::st_cluster_v4(rbase + (uint32_t)(c4 * 128 + row) * 16u, v[4 * i4],
+                               v[4 * i4 + 1], v[4 * i4 + 2], v[4 * i4 + 3]);
+          }
+        }
+      }
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();   // the partials have landed
+    ptx::tc_fence_after();
+    if (warp < 8 && role < 3 && (warp & 3) < quads_used) {
+      // the owner: its own partial plus the three received ones, in the
+      // order of the senders' ranks, back into its TMEM columns
+      const int quad = warp & 3, hh = warp >> 2;
+      const int row = quad * 32 + lane;
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        float v[32];
+        const uint32_t col = trow + 128 * role + 64 * hh + 32 * j;
+        ptx::tmem_ld32(col, v);
+        ptx::tmem_ld_wait();
+#pragma unroll 1
+        for (int sl = 0; sl < 3; ++sl) {
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const int c4 = 16 * hh + 8 * j + i4;
+            const float4 p4 = *reinterpret_cast<const float4*>(
+                smem + sl * CL_SLOT_BYTES + (c4 * 128 + row) * 16);
+            v[4 * i4] += p4.x;
+            v[4 * i4 + 1] += p4.y;
+            v[4 * i4 + 2] += p4.z;
+            v[4 * i4 + 3] += p4.w;
+          }
+        }
+        ptx::tmem_st32(col, v);
+      }
+      ptx::tmem_st_wait();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+  }
   {
     const int quad = warp & 3;
     const int i = quad * 32 + lane;
@@ -791,13 +868,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp >= 8) {
       // producer and MMA warps take no part in the epilogue
     } else if (kSplit) {
-      if (role == 0 && warp < 4)
-        epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF);
-      else if (role == 1 && warp >= 4)
-        epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF);
+      // the owner's block, warp half c taking dimensions [32c, 32c + 32)
+      // and their rotate-half partners
+      const int c = warp >> 2;
+      if (role == 0)
+        epi_q(trow + 0, ctrl->row_q[i], valid, pos, a.rope_cos, a.rope_sin, smem + Q_OFF, c, c + 1);
+      else if (role == 1)
+        epi_kv(trow + 128, i, valid, true, pos, a.rope_cos, a.rope_sin, smem + KST_OFF, c, c + 1);
       else if (role == 2)
-        epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF,
-               warp < 4 ? 0 : 1, warp < 4 ? 1 : 2);
+        epi_kv(trow + 256, i, valid, false, pos, a.rope_cos, a.rope_sin, smem + VST_OFF, c, c + 1);
     } else {
       // warp half c: q and k of dimensions [32c, 32c + 32) (+ partners),
       // then the v pass c
@@ -819,7 +898,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int r = idx >> 5;
       const int part = idx & 31;
       const int ch = part & 15;
-      if (kSplit && (role == 0 || (role == 1) != (part < 16))) continue;
+      if (kSplit && (role == 0 || role == 3 || (role == 1) != (part < 16))) continue;
       const int page = ctrl->row_page[r];
       if (page < 0) continue;
       const int slot = ctrl->row_slot[r];
@@ -835,19 +914,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   asm volatile("fence.proxy.async.global;" ::: "memory");
   fence_async_smem();
   if constexpr (kSplit) {
-    // k/v writers: every thread's cache stores, then the flag (release)
+    // k / v owners: every thread's cache stores, then one arrival (release,
+    // cluster scope) on rank 0's kv_ready. A test can withhold the arrivals
+    // (split_wait_epoch != split_epoch), so that rank 0's bounded wait runs
+    // out.
     __threadfence();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    uint32_t* flag = a.split_flags + 2 * tile_id;
-    if (role != 0 && tid == 0) ptx::st_release_gpu(flag + (role - 1), a.split_epoch);
-    // q CTA: both flags (acquire), then the cache is read through TMA
+    if ((role == 1 || role == 2) && tid == 0 && a.split_wait_epoch == a.split_epoch)
+      ptx::mbar_arrive_remote(ptx::mapa_shared(ptx::smem_u32(&ctrl->kv_ready), 0u));
+    // rank 0: both arrivals (acquire), then the cache is read through TMA
     if (role == 0 && tid == 0) {
-      bool ok = true;
-      for (int f = 0; f < 2 && ok; ++f)
-        ok = ptx::wait_flag_gpu(flag + f, a.split_wait_epoch, a.flag_wait_ns);
-      if (!ok) {
+      if (!ptx::mbar_wait_cluster(&ctrl->kv_ready, 0, a.flag_wait_ns)) {
         set_err(a.err, kDevTimeout, 30);
         atomicExch(&ctrl->abort, 1);
       }
@@ -866,10 +945,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t pt_base = ptx::smem_u32(smem + PT_OFF);
   const uint32_t qrep_base = ptx::smem_u32(smem + QREP_OFF);
 
-  // k/v CTAs of a split tile stop here, and so does an attending CTA whose
-  // wait for them gave up: it issues no load and no product, so nothing is
-  // left in flight (its out rows stay unwritten, its mass partials zero, and
-  // the error word holds the timeout)
+  // ranks 1-3 of a split tile stop here, and so does rank 0 when its wait
+  // for the k / v owners gave up: it issues no load and no product, so
+  // nothing is left in flight (its out rows stay unwritten, its mass
+  // partials zero, and the error word holds the timeout)
   const bool gave_up = kSplit && *reinterpret_cast<volatile int*>(&ctrl->abort) != 0;
   const int nseq_g = (role == 0 && !gave_up) ? ctrl->nseq : 0;
   auto seq_resident = [&](int q) -> bool {
@@ -1569,7 +1648,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    kstep0 += nkb;
+    kstep0 += kb1 - kb0;
   }
   }   // tiles
 
@@ -1577,42 +1656,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, TMEM_COLS);
+  // no rank leaves while another may still arrive on its shared memory
+  if constexpr (kSplit) ptx::cluster_sync();
 }
 
 template <bool kPersist, bool kSplit, typename Sched>
 cudaError_t launch_kernel(int grid, const StepPlan& plan, const Sched& sched, const StepArgs& a,
-                          const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
-                          const void* tmap_k, const void* tmap_v, cudaStream_t stream) {
+                          const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                          const void* tmap_v, cudaStream_t stream) {
   static std::atomic<uint64_t> attr_done{0};
   cudaError_t e = opt_in_smem(reinterpret_cast<const void*>(step_bf16_kernel<kPersist, kSplit>),
                               SMEM_BYTES, attr_done);
   if (e != cudaSuccess) return e;
-  step_bf16_kernel<kPersist, kSplit><<<grid, NTHREADS, SMEM_BYTES, stream>>>(
-      plan, sched, a, *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_x[1]), *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
-      *reinterpret_cast<const CUtensorMap*>(tmap_w), *reinterpret_cast<const CUtensorMap*>(tmap_w1),
-      *reinterpret_cast<const CUtensorMap*>(tmap_k), *reinterpret_cast<const CUtensorMap*>(tmap_v));
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (kSplit) {   // one cluster of CL_RANKS CTAs per tile
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL_RANKS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, step_bf16_kernel<kPersist, kSplit>, plan, sched, a,
+                            *reinterpret_cast<const CUtensorMap*>(tmap_x[0]),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_x[1]),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_x[2]),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_x[3]),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_w),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_k),
+                            *reinterpret_cast<const CUtensorMap*>(tmap_v));
 }
 
 }  // namespace
 
 size_t step_bf16_smem_bytes() { return SMEM_BYTES; }
 
+bool step_bf16_split_ok(int tiles, int hidden, int sms) {
+  return tiles > 0 && sms > 0 && CL_RANKS * tiles <= sms && hidden % (CL_RANKS * BK) == 0;
+}
+
 cudaError_t launch_step_bf16(const StepPlan& plan, const TileSched& sched, const StepArgs& a,
-                             const void* const* tmap_x, const void* tmap_w, const void* tmap_w1,
-                             const void* tmap_k, const void* tmap_v, cudaStream_t stream) {
+                             const void* const* tmap_x, const void* tmap_w, const void* tmap_k,
+                             const void* tmap_v, bool split, cudaStream_t stream) {
   if (sched.n_bins > 0)
-    return launch_kernel<true, false>(sched.n_bins, plan, sched, a, tmap_x, tmap_w, tmap_w,
-                                      tmap_k, tmap_v, stream);
+    return launch_kernel<true, false>(sched.n_bins, plan, sched, a, tmap_x, tmap_w, tmap_k,
+                                      tmap_v, stream);
   const int grid = plan.n_groups * a.n_heads;
   if (grid == 0) return cudaSuccess;
-  if (a.split_flags && tmap_w1)
-    return launch_kernel<false, true>(3 * grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_w1,
+  if (split)
+    return launch_kernel<false, true>(CL_RANKS * grid, plan, NoSched{0}, a, tmap_x, tmap_w,
                                       tmap_k, tmap_v, stream);
-  return launch_kernel<false, false>(grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_w, tmap_k,
-                                     tmap_v, stream);
+  return launch_kernel<false, false>(grid, plan, NoSched{0}, a, tmap_x, tmap_w, tmap_k, tmap_v,
+                                     stream);
 }
 
 }  // namespace fdllm

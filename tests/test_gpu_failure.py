@@ -3,9 +3,10 @@ to run out by a host-side injection, the step reports FDLLM_ERR_TIMEOUT
 through fdllm_check, and the same handle then runs a correct step.
 
 The injected wait is the one that the attending CTA of a split tile makes
-for the two cache-writing CTAs of its tile (small steps split each tile over
-three CTAs). The injection makes it wait for a flag value nobody stores,
-bounded to a few milliseconds; nothing traps, faults or spins unbounded."""
+for the two cache-writing CTAs of its cluster (small steps run each tile as
+a cluster of four CTAs). The injection makes those CTAs withhold their
+signal, and the wait is bounded to a few milliseconds; nothing traps,
+faults or spins unbounded."""
 import numpy as np
 import pytest
 import torch
@@ -34,7 +35,7 @@ def test_injected_flag_wait_times_out_and_the_handle_recovers():
     fd.fdllm_inject_fault(cache.handle, _lib.FDLLM_INJECT_SPLIT_FLAG_TIMEOUT, 2_000_000)
     cache.step(0, meta.cu_rows, meta.seq_lens, x.to(dev), w.to(dev), pos, bt, view_mask=view,
                slots=slots, validate=False)
-    # this step's tiles were split over three CTAs (the injection is used up)
+    # this step's tiles ran as four-CTA clusters (the injection is used up)
     with pytest.raises(fd.FdllmError) as ei:
         cache.check()
     assert ei.value.status == _lib.FDLLM_ERR_TIMEOUT
