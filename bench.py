@@ -68,10 +68,10 @@ def load_peaks():
 # that plans its launch. The figure is reported only while all three match.
 CAPTURED_TRAFFIC = {
     "b32_divergent": {
-        "bytes": 783267072.0,     # 724.95 MB read + 58.32 MB written, one launch
-        "sources": ["74dc2982d14adbcae91472b3f5ed01e311929a173c789f70c1e5573ed147451b",
-                    "be391d302227a2ef2fe5128f6ea54d3e927a312868f880e0d405437ecf91a423",
-                    "f8854e1e241ad568d316e6e6ccbd4e206f5d57ddd64b5c73740d61d765e7ef10"],
+        "bytes": 746224896.0,     # 695.71 MB read + 50.51 MB written, one launch
+        "sources": ["613eb139d9c12733527256ba55743b3103bf4c601f119db75cf6dbfd62813bc0",
+                    "fe252cfc00f64efb448b0b58ddb2084b317046d35d5a39eef1fab7842009c83a",
+                    "552a823d86a5e54df26e2e180d35ea47c9a07907f4669983f5435c1b5c152123"],
         "source": "ncu --set full, one launch (profiles/step_bf16_b32_divergent.md)",
     },
 }
