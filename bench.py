@@ -29,6 +29,7 @@ One JSON line is printed by rank 0.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -1300,9 +1301,19 @@ def main(argv=None):
                     help="unfused arm: skip counting its kernels with the torch profiler")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the table of the other layer workloads in the default run")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="run a layer workload with this many layers (same per-layer shapes and "
+                         "contexts; a small case of a deep stack for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.layers is not None:
+        if args.workload not in W.WORKLOADS or args.layers < 1:
+            ap.error("--layers takes a positive count and a layer workload")
+        s = W.WORKLOADS[args.workload]
+        W.WORKLOADS[args.workload] = dataclasses.replace(
+            s, shape=dataclasses.replace(s.shape, n_layers=args.layers))
+        args.no_per_workload = True
     if args.workload in W.VERIFY_WORKLOADS:
         return run_verify(args)
     if args.workload in W.OPROJ_WORKLOADS:
