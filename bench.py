@@ -1310,10 +1310,19 @@ def main(argv=None):
     if args.layers is not None:
         if args.workload not in W.WORKLOADS or args.layers < 1:
             ap.error("--layers takes a positive count and a layer workload")
+        # the named workload with another layer count, for this run only
         s = W.WORKLOADS[args.workload]
         W.WORKLOADS[args.workload] = dataclasses.replace(
             s, shape=dataclasses.replace(s.shape, n_layers=args.layers))
         args.no_per_workload = True
+        try:
+            return _dispatch(args)
+        finally:
+            W.WORKLOADS[args.workload] = s
+    return _dispatch(args)
+
+
+def _dispatch(args):
     if args.workload in W.VERIFY_WORKLOADS:
         return run_verify(args)
     if args.workload in W.OPROJ_WORKLOADS:

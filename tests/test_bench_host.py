@@ -48,3 +48,24 @@ def test_reference_arm_times_whole_sampled_steps(capsys):
     assert line["impl"] == "reference"
     assert line["ms_per_step"] * line["steps"] / 1000.0 <= wall
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_layers_option_changes_the_layer_count_for_one_run(capsys):
+    """--layers runs a layer workload with another layer count (the same
+    per-layer shapes) and leaves the workload table as it was."""
+    import json
+
+    import pytest
+
+    from kv_cache_attention_flash_b200 import workloads as W
+    before = W.WORKLOADS["tiny_f32"]
+    assert bench.main(["--impl", "reference", "--workload", "tiny_f32", "--layers", "2",
+                       "--steps", "3", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"]["layers"] == 2
+    assert line["config"]["hidden"] == before.shape.hidden
+    assert W.WORKLOADS["tiny_f32"] is before
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "tiny_f32", "--layers", "0"])
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "verify_b8", "--layers", "1"])
