@@ -69,11 +69,12 @@ def load_peaks():
 # that plans its launch. The figure is reported only while all three match.
 CAPTURED_TRAFFIC = {
     "b32_divergent": {
-        "bytes": 746224896.0,     # 695.71 MB read + 50.51 MB written, one launch
-        "sources": ["613eb139d9c12733527256ba55743b3103bf4c601f119db75cf6dbfd62813bc0",
+        "bytes": 737150208.0,     # 685.69 MB read + 51.46 MB written, one launch
+        "sources": ["b33b07c2690a533491b3ff6b70bfd4feaf46421e59324abb29403571b548df37",
                     "fe252cfc00f64efb448b0b58ddb2084b317046d35d5a39eef1fab7842009c83a",
                     "552a823d86a5e54df26e2e180d35ea47c9a07907f4669983f5435c1b5c152123"],
-        "source": "ncu --set full, one launch (profiles/step_bf16_b32_divergent.md)",
+        "source": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum, one launch "
+                  "(profiles/step_bf16_b32_divergent.md)",
     },
 }
 

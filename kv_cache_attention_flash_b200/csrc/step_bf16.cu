@@ -321,22 +321,29 @@ __device__ __forceinline__ void epi_qk(uint32_t trow, int c, int qrow, int row, 
 // (raw S values; the scale sl2 = log2(e)/sqrt(D) is applied in the
 // exponent's FMA). Keys whose bit in mk is clear are dropped before
 // anything else, so a NaN in an unattended slot never reaches the sums.
-// Four independent max / sum chains.
+// Eight independent max / sum chains.
 template <int NK>
-__device__ __forceinline__ void lse_block(float* v, uint32_t mk, float sl2, float& m, float& l) {
-  float b4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+__device__ __forceinline__ void lse_block(float* v, uint64_t mk, float sl2, float& m, float& l) {
+  float b8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b8[i] = -INFINITY;
 #pragma unroll
   for (int j = 0; j < NK; ++j) {
-    v[j] = ((mk >> j) & 1u) ? v[j] : -INFINITY;
-    b4[j & 3] = fmaxf(b4[j & 3], v[j]);
+    v[j] = ((mk >> j) & 1ull) ? v[j] : -INFINITY;
+    b8[j & 7] = fmaxf(b8[j & 7], v[j]);
   }
   // rounding is monotone, so the scaled maximum is the maximum scaled score
-  const float mn = fmaxf(m, fmaxf(fmaxf(b4[0], b4[1]), fmaxf(b4[2], b4[3])) * sl2);
+  const float bm = fmaxf(fmaxf(fmaxf(b8[0], b8[1]), fmaxf(b8[2], b8[3])),
+                         fmaxf(fmaxf(b8[4], b8[5]), fmaxf(b8[6], b8[7])));
+  const float mn = fmaxf(m, bm * sl2);
   if (mn == -INFINITY) return;
-  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  float s8[8];
 #pragma unroll
-  for (int j = 0; j < NK; ++j) s4[j & 3] += ptx::ex2(fmaf(v[j], sl2, -mn));
-  l = l * ptx::ex2(m - mn) + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+  for (int i = 0; i < 8; ++i) s8[i] = 0.f;
+#pragma unroll
+  for (int j = 0; j < NK; ++j) s8[j & 7] += ptx::ex2(fmaf(v[j], sl2, -mn));
+  l = l * ptx::ex2(m - mn) +
+      (((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7])));
   m = mn;
 }
 
@@ -1421,43 +1428,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < nch; ++c) {
           const uint32_t idx = s0 + c;
           const uint32_t sb = idx & 1;
+          // This thread's keys [jbeg, jbeg + KH) of the chunk lie in one
+          // page, pidx (KH = 64, 32 or 16 and jbeg a multiple of KH); its
+          // row attends the page's context slots, then view slots of its
+          // own view at positions <= its own. The mask is formed before
+          // the scores are waited for.
+          uint64_t km = 0ull;
+          if (warp_active) {
+            const int pidx = 2 * c + (jbeg >> 6);
+            if (active && pidx < npages && pgp[pidx] >= 0) {
+              const int plog = (int)pgl[pidx];
+              const int nv = min(max(L - plog * PS, 0), PS);
+              km = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
+              if (nv < PS && myview != 0) {
+                for (int x = 0; x < nx; ++x) {
+                  const int xs = xsl[x];
+                  const int xr = xsr[x];
+                  if (xs / PS == plog && ctrl->row_view[xr] == myview &&
+                      ctrl->row_pos[xr] <= mypos)
+                    km |= 1ull << (xs % PS);
+                }
+              }
+              km >>= (jbeg & 63);
+            }
+          }
           wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 20);
           ptx::tc_fence_after();
           if (warp_active) {
-#pragma unroll 1
-            for (int j0 = jbeg; j0 < jbeg + KH; j0 += 32) {
-              const int nk = KH < 32 ? KH : 32;      // keys in this block (16 or 32)
-              // keys j0 .. j0+nk-1 of the chunk lie in one page, pidx; this
-              // row attends its context slots, then view slots of its own
-              // view at positions <= its own
-              const int pidx = 2 * c + (j0 >> 6);
-              uint64_t km = 0ull;
-              if (pidx < npages && pgp[pidx] >= 0) {
-                const int plog = (int)pgl[pidx];
-                const int nv = min(max(L - plog * PS, 0), PS);
-                km = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);
-                if (nv < PS && myview != 0) {
-                  for (int x = 0; x < nx; ++x) {
-                    const int xs = xsl[x];
-                    const int xr = xsr[x];
-                    if (xs / PS == plog && ctrl->row_view[xr] == myview &&
-                        ctrl->row_pos[xr] <= mypos)
-                      km |= 1ull << (xs % PS);
-                  }
-                }
-              }
-              const uint32_t mk = active ? (uint32_t)(km >> (j0 & 63)) : 0u;
+            const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + jbeg;
+            if (KH == 64) {
+              // both loads in flight before the one wait
+              float v[64];
+              ptx::tmem_ld32(sbase, v);
+              ptx::tmem_ld32(sbase + 32, v + 32);
+              ptx::tmem_ld_wait();
+              lse_block<64>(v, km, sl2, m, l);
+            } else if (KH == 32) {
               float v[32];
-              const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + j0;
-              if (nk == 32) {
-                ptx::tmem_ld32(sbase, v);
-                ptx::tmem_ld_wait();
-                lse_block<32>(v, mk, sl2, m, l);
-              } else {
-                ptx::tmem_ld16(sbase, v);
-                ptx::tmem_ld_wait();
-                lse_block<16>(v, mk, sl2, m, l);
-              }
+              ptx::tmem_ld32(sbase, v);
+              ptx::tmem_ld_wait();
+              lse_block<32>(v, km, sl2, m, l);
+            } else {
+              float v[16];
+              ptx::tmem_ld16(sbase, v);
+              ptx::tmem_ld_wait();
+              lse_block<16>(v, km, sl2, m, l);
             }
           }
           ptx::tc_fence_before();
@@ -1488,69 +1503,83 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
       // ----- pass 2: probabilities, mass, P^T for the P.V product. S^T has
       // the chunk's keys on TMEM lanes (thread t owns key t) and this
-      // sequence's rows on columns; the warp pair splits the rows in
-      // 16-row sub-blocks (sub-block k goes to half k % 2).
-      const int nsub = N16 >> 4;
+      // sequence's rows on columns; warp half `half` takes the NC = N16 / 2
+      // rows [half * NC, half * NC + NC). Its scores are loaded (at most two
+      // 32-column loads in flight) while the previous chunk's P.V product
+      // may still be reading the single P^T buffer; once both are done the
+      // TMEM buffer is released and P^T is written eight rows at a time.
+      const int NC = N16 >> 1;
+      const int c0 = half * NC;
+      // visibility of this thread's key to the rows [c0, c0 + 64), bit j for row c0 + j
+      auto vis_bits = [&](int cat, int xr) -> uint64_t {
+        if (cat == 0) return 0ull;
+        const int lim = n - c0;
+        if (cat == 1) return lim >= 64 ? ~0ull : (lim <= 0 ? 0ull : ((1ull << lim) - 1ull));
+        const int kv = ctrl->row_view[xr], kp = ctrl->row_pos[xr];
+        uint64_t m = 0ull;
+        for (int j = 0; j < 64 && j < lim; ++j) {
+          const int rr = ra + c0 + j;
+          if (ctrl->row_view[rr] == kv && ctrl->row_pos[rr] >= kp) m |= 1ull << j;
+        }
+        return m;
+      };
       for (int c = 0; c < nch; ++c) {
         int slot, cat, xr;
         key_info(c, slot, cat, xr);
+        const uint64_t vm = vis_bits(cat, xr);
         const int pidx = 2 * c + (t >> 6);
         const bool loaded = pidx < npages && pgp[pidx] >= 0;
         const uint32_t idx = s0 + nch + c;
         const uint32_t sb = idx & 1;
         wait_bar(ctrl, &ctrl->s_full[sb], (idx >> 1) & 1, a.err, 21);
         ptx::tc_fence_after();
-        const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0);
+        const uint32_t sbase = tmem + tl + (sb ? TM_S1 : TM_S0) + (uint32_t)c0;
+        float v[64];
+        ptx::tmem_ld32(sbase, v);
+        if (NC > 32) ptx::tmem_ld32(sbase + 32, v + 32);
         // The P^T buffer is free once the previous P.V product completed
         // (pv_done counts the two-pass chunks only; earlier resident chunks'
         // products completed before this sequence began, at that sequence's
-        // o_done). P^T is then written eight rows at a time.
+        // o_done).
         const uint32_t pidx_g = opcount + c;
         if (pidx_g > 0) wait_bar(ctrl, &ctrl->pv_done, (pidx_g - 1) & 1, a.err, 23);
+        ptx::tmem_ld_wait();
+        // the scores are in registers: the TMEM buffer can take S^T of chunk c + 2
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
         uint8_t* pth = smem + PT_OFF;
         uint8_t* ptl = pth + ptl_off;
         float mass2[2] = {0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int k = 2 * u + half;            // 16-row sub-block
-          if (k < nsub) {
-            const uint32_t m16 = (vis_mask(cat, xr, k >> 1) >> (16 * (k & 1))) & 0xffffu;
-            float v[16];
-            ptx::tmem_ld16(sbase + 16 * k, v);
-            const float4* l4 = reinterpret_cast<const float4*>(ctrl->lse2 + 16 * k);
-            ptx::tmem_ld_wait();
+        for (int g8 = 0; g8 < 8; ++g8) {
+          if (8 * g8 < NC) {
+            const float4* l4 = reinterpret_cast<const float4*>(ctrl->lse2 + c0 + 8 * g8);
+            uint32_t ph[4], pq[4];
 #pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
-              uint32_t ph[4], pq[4];
-#pragma unroll
-              for (int jj = 0; jj < 2; ++jj) {
-                const int j4 = 2 * g8 + jj;
-                const float4 ll = l4[j4];
-                const int j = 4 * j4;
-                const float e0 = ptx::ex2(fmaf(v[j], sl2, -ll.x));
-                const float e1 = ptx::ex2(fmaf(v[j + 1], sl2, -ll.y));
-                const float e2 = ptx::ex2(fmaf(v[j + 2], sl2, -ll.z));
-                const float e3 = ptx::ex2(fmaf(v[j + 3], sl2, -ll.w));
-                const float q0 = ((m16 >> j) & 1u) ? e0 : 0.f;
-                const float q1 = ((m16 >> (j + 1)) & 1u) ? e1 : 0.f;
-                const float q2 = ((m16 >> (j + 2)) & 1u) ? e2 : 0.f;
-                const float q3 = ((m16 >> (j + 3)) & 1u) ? e3 : 0.f;
-                mass2[j4 & 1] += (q0 + q1) + (q2 + q3);
-                ptx::split_bf16(q0, q1, ph[2 * jj], pq[2 * jj]);
-                ptx::split_bf16(q2, q3, ph[2 * jj + 1], pq[2 * jj + 1]);
-              }
-              const int nb = 2 * k + g8;     // 8-row block of the sequence
-              *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-              *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+            for (int jj = 0; jj < 2; ++jj) {
+              const float4 ll = l4[jj];
+              const int j = 8 * g8 + 4 * jj;
+              const float e0 = ptx::ex2(fmaf(v[j], sl2, -ll.x));
+              const float e1 = ptx::ex2(fmaf(v[j + 1], sl2, -ll.y));
+              const float e2 = ptx::ex2(fmaf(v[j + 2], sl2, -ll.z));
+              const float e3 = ptx::ex2(fmaf(v[j + 3], sl2, -ll.w));
+              const float q0 = ((vm >> j) & 1ull) ? e0 : 0.f;
+              const float q1 = ((vm >> (j + 1)) & 1ull) ? e1 : 0.f;
+              const float q2 = ((vm >> (j + 2)) & 1ull) ? e2 : 0.f;
+              const float q3 = ((vm >> (j + 3)) & 1ull) ? e3 : 0.f;
+              mass2[jj] += (q0 + q1) + (q2 + q3);
+              ptx::split_bf16(q0, q1, ph[2 * jj], pq[2 * jj]);
+              ptx::split_bf16(q2, q3, ph[2 * jj + 1], pq[2 * jj + 1]);
             }
+            const int nb = (c0 >> 3) + g8;     // 8-row block of the sequence
+            *reinterpret_cast<uint4*>(pth + nb * 2048 + t * 16) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+            *reinterpret_cast<uint4*>(ptl + nb * 2048 + t * 16) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
           }
         }
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&ctrl->s_empty[sb]);
         // both halves add into the zeroed mass row; two addends, so the
         // result does not depend on their order
-        if (part && cat != 0 && nsub > half) atomicAdd(part + slot, mass2[0] + mass2[1]);
+        if (part && cat != 0) atomicAdd(part + slot, mass2[0] + mass2[1]);
         // V rows of keys nobody attends may hold anything (page tails):
         // zero them so that 0 * V stays 0 in the P.V product (each half
         // clears one 64-dimension half of the row).
