@@ -135,6 +135,8 @@ struct Ctrl {
   int sq_npages[MAX_SEQ], sq_pg0[MAX_SEQ], sq_x0[MAX_SEQ], sq_nx[MAX_SEQ], sq_any[MAX_SEQ];
   int xs_slot[BM];        // per sequence: slots written by its view rows, ascending
   int xs_row[BM];         //   and the group rows that write them
+  uint32_t xs_mask[BM][4];  //   and the rows of the sequence that see each of them
+                            //   (bit j of word w: row 32 w + j)
   short pg_log[MAX_PAGES];  // per sequence: logical pages attended, in order
   int pg_phys[MAX_PAGES];   //   and their physical pages (-1: bad table entry)
   alignas(16) float lse2[BM];   // log2-sum-exp2 of the scaled scores of each row (float4 loads)
@@ -712,6 +714,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ctrl->xs_row[ctrl->sq_x0[q] + rank] = i;
     }
     named_bar(2, NM);
+    // Flash-Verify visibility of each view slot, once per tile: row rr of
+    // its sequence sees the slot written by row xr when both are of the
+    // same view and rr's position is not before xr's
+    {
+      const int nxs = nseq > 0 ? ctrl->sq_x0[nseq - 1] + ctrl->sq_nx[nseq - 1] : 0;
+      for (int it = mt; it < nxs * 4; it += NM) {
+        const int x = it >> 2, w = it & 3;
+        int q = 0;
+        while (q + 1 < nseq && ctrl->sq_x0[q + 1] <= x) ++q;
+        const int xr = ctrl->xs_row[x];
+        const int kv = ctrl->row_view[xr], kp = ctrl->row_pos[xr];
+        uint32_t m = 0u;
+        for (int j = 0; j < 32; ++j) {
+          const int col = 32 * w + j;
+          if (col < ctrl->sq_n[q]) {
+            const int rr = ctrl->sq_qoff[q] + col;
+            if (ctrl->row_view[rr] == kv && ctrl->row_pos[rr] >= kp) m |= 1u << j;
+          }
+        }
+        ctrl->xs_mask[x][w] = m;
+      }
+    }
+    named_bar(2, NM);
     // logical pages: the context pages, then the pages of view slots past them
     if (mt < nseq) {
       const int npr = (ctrl->sq_L[mt] + PS - 1) / PS;
@@ -976,7 +1001,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const short* pgl = ctrl->pg_log + ctrl->sq_pg0[si];
     const int* pgp = ctrl->pg_phys + ctrl->sq_pg0[si];
     const int* xsl = ctrl->xs_slot + ctrl->sq_x0[si];
-    const int* xsr = ctrl->xs_row + ctrl->sq_x0[si];
     const int nch = (npages + 1) >> 1;
     // Resident scores (a sequence of 16, 32 or 64 padded rows whose chunks
     // fit TMEM): one S^T = K Q^T product per chunk into its own TMEM
@@ -1205,11 +1229,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int half = warp >> 2;
       const int t = quad * 32 + lane;
       const uint32_t tl = (uint32_t)(quad * 32) << 16;
-      // cat: 0 nobody attends the key, 1 every row does, 2 a view row's slot
-      auto key_info = [&](int c, int& slot, int& cat, int& xr) {
+      // cat: 0 nobody attends the key, 1 every row does, 2 a view row's
+      // slot (xi: its index among the sequence's view slots)
+      auto key_info = [&](int c, int& slot, int& cat, int& xi) {
         const int pidx = 2 * c + (t >> 6);
         cat = 0;
-        xr = -1;
+        xi = -1;
         slot = -1;
         if (pidx >= npages || pgp[pidx] < 0) return;
         slot = (int)pgl[pidx] * PS + (t & 63);
@@ -1223,7 +1248,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int v = xsl[mid];
           if (v == slot) {
             cat = 2;
-            xr = xsr[mid];
+            xi = mid;
             return;
           }
           if (v < slot) lo = mid + 1; else hi = mid - 1;
@@ -1231,21 +1256,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       // Visibility of this thread's key to the 32 rows [32*blk, 32*blk+32)
       // of the sequence, as a bit mask.
-      auto vis_mask = [&](int cat, int xr, int blk) -> uint32_t {
+      const uint32_t (*xsm)[4] = ctrl->xs_mask + ctrl->sq_x0[si];
+      auto vis_mask = [&](int cat, int xi, int blk) -> uint32_t {
         if (cat == 0) return 0u;
-        const int lim = n - 32 * blk;
-        const uint32_t rows = lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
-        if (cat == 1) return rows;
-        const int kv = ctrl->row_view[xr], kp = ctrl->row_pos[xr];
-        uint32_t m = 0u;
-        for (int j = 0; j < 32; ++j) {
-          const int col = 32 * blk + j;
-          if (col < n) {
-            const int rr = ra + col;
-            if (ctrl->row_view[rr] == kv && ctrl->row_pos[rr] >= kp) m |= 1u << j;
-          }
+        if (cat == 1) {
+          const int lim = n - 32 * blk;
+          return lim >= 32 ? 0xffffffffu : (lim <= 0 ? 0u : ((1u << lim) - 1u));
         }
-        return m;
+        return xsm[xi][blk];
       };
 
       // ----- resident scores (see above). Thread t owns key t of every
@@ -1257,9 +1275,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int rbase = half * NR;
         const uint32_t cbase = tmem + tl + (uint32_t)rbase;
         auto row_mask = [&](int c, int& slot, int& cat) -> uint32_t {
-          int xr;
-          key_info(c, slot, cat, xr);
-          const uint32_t m = vis_mask(cat, xr, rbase >> 5) >> (rbase & 31);
+          int xi;
+          key_info(c, slot, cat, xi);
+          const uint32_t m = vis_mask(cat, xi, rbase >> 5) >> (rbase & 31);
           return NR == 32 ? m : (m & ((1u << NR) - 1u));
         };
         float acc[32];
@@ -1421,7 +1439,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const bool active = r >= 0 && r < n;
         const bool warp_active = __any_sync(0xffffffffu, active);
         const int myview = active ? ctrl->row_view[ra + r] : 0;
-        const int mypos = active ? ctrl->row_pos[ra + r] : 0;
         const int KH = KR >> 1;                      // keys per thread per chunk
         const int jbeg = rho * KR + half * KH;       // first chunk column of this thread
         float m = -INFINITY, l = 0.f;
@@ -1443,9 +1460,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (nv < PS && myview != 0) {
                 for (int x = 0; x < nx; ++x) {
                   const int xs = xsl[x];
-                  const int xr = xsr[x];
-                  if (xs / PS == plog && ctrl->row_view[xr] == myview &&
-                      ctrl->row_pos[xr] <= mypos)
+                  if (xs / PS == plog && ((xsm[x][r >> 5] >> (r & 31)) & 1u))
                     km |= 1ull << (xs % PS);
                 }
               }
@@ -1511,22 +1526,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int NC = N16 >> 1;
       const int c0 = half * NC;
       // visibility of this thread's key to the rows [c0, c0 + 64), bit j for row c0 + j
-      auto vis_bits = [&](int cat, int xr) -> uint64_t {
+      auto vis_bits = [&](int cat, int xi) -> uint64_t {
         if (cat == 0) return 0ull;
         const int lim = n - c0;
         if (cat == 1) return lim >= 64 ? ~0ull : (lim <= 0 ? 0ull : ((1ull << lim) - 1ull));
-        const int kv = ctrl->row_view[xr], kp = ctrl->row_pos[xr];
-        uint64_t m = 0ull;
-        for (int j = 0; j < 64 && j < lim; ++j) {
-          const int rr = ra + c0 + j;
-          if (ctrl->row_view[rr] == kv && ctrl->row_pos[rr] >= kp) m |= 1ull << j;
-        }
-        return m;
+        const int w = c0 >> 5, sh = c0 & 31;
+        const uint64_t lo = (uint64_t)xsm[xi][w] | ((w + 1 < 4 ? (uint64_t)xsm[xi][w + 1] : 0ull) << 32);
+        const uint64_t hi = w + 2 < 4 ? (uint64_t)xsm[xi][w + 2] : 0ull;
+        return sh == 0 ? lo : ((lo >> sh) | (hi << (64 - sh)));
       };
       for (int c = 0; c < nch; ++c) {
-        int slot, cat, xr;
-        key_info(c, slot, cat, xr);
-        const uint64_t vm = vis_bits(cat, xr);
+        int slot, cat, xi;
+        key_info(c, slot, cat, xi);
+        const uint64_t vm = vis_bits(cat, xi);
         const int pidx = 2 * c + (t >> 6);
         const bool loaded = pidx < npages && pgp[pidx] >= 0;
         const uint32_t idx = s0 + nch + c;
