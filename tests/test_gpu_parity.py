@@ -289,6 +289,61 @@ def test_edge_cases_empty_and_maximal_sequences():
     assert np.allclose(g.mass[[0, 2, 3]].sum(1), 1.0, atol=1e-5)
 
 
+def _two_view_meta(specs, seed):
+    """A step of two-view sequences: each (L, n_v, interleave) gives a
+    context of L slots and two views of n_v rows at positions L .. L+n_v-1,
+    view 1 writing slots L .. L+n_v-1 and view 2 the next n_v slots;
+    interleave alternates the two views' rows."""
+    rng = np.random.default_rng(seed)
+    ps = 64
+    rows, lens, nblk = [], [], []
+    for L, nv, inter in specs:
+        pos = np.arange(L, L + nv)
+        p = np.concatenate([pos, pos])
+        sl = np.concatenate([np.arange(L, L + nv), np.arange(L + nv, L + 2 * nv)])
+        v = np.concatenate([np.ones(nv, np.int8), np.full(nv, 2, np.int8)])
+        if inter:
+            order = np.stack([np.arange(nv), np.arange(nv, 2 * nv)], 1).reshape(-1)
+            p, sl, v = p[order], sl[order], v[order]
+        rows.append((p, sl, v))
+        lens.append(L)
+        nblk.append((L + 2 * nv + ps - 1) // ps)
+    batch = len(specs)
+    npg = sum(nblk) + 3
+    perm = rng.permutation(npg)
+    bt = np.full((batch, max(nblk)), -1, np.int32)
+    k = 0
+    for b in range(batch):
+        for i in range(nblk[b]):
+            bt[b, i] = perm[k]
+            k += 1
+    cu = np.zeros(batch + 1, np.int32)
+    cu[1:] = np.cumsum([len(r[0]) for r in rows])
+    return W.StepMeta(batch=batch, cu_rows=cu, seq_lens=np.array(lens, np.int32),
+                      positions=np.concatenate([r[0] for r in rows]).astype(np.int32),
+                      slots=np.concatenate([r[1] for r in rows]).astype(np.int32),
+                      view=np.concatenate([r[2] for r in rows]).astype(np.int8), block_table=bt,
+                      num_pages=npg, max_position=max(L + nv for L, nv, _ in specs) + 1,
+                      exclude_cu=np.zeros(batch + 1, np.int32),
+                      exclude_slots=np.zeros(0, np.int32), track_k=8,
+                      stage=np.zeros(batch, np.int8))
+
+
+def test_two_view_masks_in_every_attention_shape():
+    """Fresh view keys in every attention form: resident scores with 16 and
+    32 padded rows (views of 4 and 16 rows), and two-pass sequences of 80 and
+    96 rows (views of 40 and 48 rows, whose warp halves start at rows 40 and
+    48), one with the two views' rows interleaved, one with 19 pages."""
+    sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
+    spec = W.WorkloadSpec("two_view_shapes", sh, batch=4, kind="divergent", ctx_min=1, ctx_max=1)
+    meta = _two_view_meta([(100, 16, False), (300, 48, True), (1100, 40, False), (20, 4, True)], 5)
+    x = W.make_x(spec, meta, 2)
+    w = W.make_w(spec, 2)
+    kp, vp = W.make_pools(spec, meta, 2, n_layers=1)
+    g = run_gpu(spec, meta, x, w, kp, vp)
+    check_dense(spec, meta, x, w, kp, vp, g)
+
+
 def test_all_rows_empty_step():
     sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
     spec = W.WorkloadSpec("empty", sh, batch=2, kind="divergent", ctx_min=1, ctx_max=1)
