@@ -331,12 +331,14 @@ def _two_view_meta(specs, seed):
 
 def test_two_view_masks_in_every_attention_shape():
     """Fresh view keys in every attention form: resident scores with 16 and
-    32 padded rows (views of 4 and 16 rows), and two-pass sequences of 80 and
-    96 rows (views of 40 and 48 rows, whose warp halves start at rows 40 and
-    48), one with the two views' rows interleaved, one with 19 pages."""
+    32 padded rows (views of 4 and 16 rows), and two-pass sequences of 80,
+    96, 112 and 128 rows (views of 40, 48, 56 and 64 rows, whose second warp
+    halves start at rows 40, 48, 56 and 64), some with the two views' rows
+    interleaved, one with 19 pages."""
     sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
-    spec = W.WorkloadSpec("two_view_shapes", sh, batch=4, kind="divergent", ctx_min=1, ctx_max=1)
-    meta = _two_view_meta([(100, 16, False), (300, 48, True), (1100, 40, False), (20, 4, True)], 5)
+    spec = W.WorkloadSpec("two_view_shapes", sh, batch=6, kind="divergent", ctx_min=1, ctx_max=1)
+    meta = _two_view_meta([(100, 16, False), (300, 48, True), (1100, 40, False), (20, 4, True),
+                           (60, 56, True), (200, 64, False)], 5)
     x = W.make_x(spec, meta, 2)
     w = W.make_w(spec, 2)
     kp, vp = W.make_pools(spec, meta, 2, n_layers=1)
