@@ -346,6 +346,30 @@ def test_two_view_masks_in_every_attention_shape():
     check_dense(spec, meta, x, w, kp, vp, g)
 
 
+def test_persistent_grid_with_every_attention_form():
+    """More tiles than SMs, so the persistent kernel runs them from its
+    schedule and carries its barrier phases and counters from tile to tile
+    through two-view sequences of all three forms: two-pass of 64 rows (19
+    pages), two-pass of 96 rows with interleaved views, resident of 32 rows.
+    On a B200: 5.9e-5 x RMS on grid inputs; 6.9e-3 on continuous ones, where
+    one-ulp differences of fresh bf16 k / v rows (fp32 against float64
+    accumulation) weigh more against the small RMS of outputs averaged over
+    1100-slot contexts."""
+    sh = W.LayerShape("bf16", 2048, 16, 128, 64, 10000.0)
+    specs = [(1100, 32, i % 2 == 1) for i in range(16)] + [(300, 48, True)] * 2 + [(500, 16, False)] * 2
+    spec = W.WorkloadSpec("persistent_views", sh, batch=len(specs), kind="divergent",
+                          ctx_min=1, ctx_max=1)
+    meta = _two_view_meta(specs, 9)
+    kp, vp = W.make_pools(spec, meta, 3, n_layers=1)
+    # continuous inputs, then inputs on which the fp32 projection is exact
+    # (written k / v bit-exact, out free of the fresh rows' rounding flips)
+    for grid in (False, True):
+        x = (W.make_x_grid if grid else W.make_x)(spec, meta, 3)
+        w = (W.make_w_grid if grid else W.make_w)(spec, 3)
+        g = run_gpu(spec, meta, x, w, kp, vp)
+        check_dense(spec, meta, x, w, kp, vp, g, grid=grid)
+
+
 def test_all_rows_empty_step():
     sh = W.LayerShape("bf16", 256, 2, 128, 64, 10000.0)
     spec = W.WorkloadSpec("empty", sh, batch=2, kind="divergent", ctx_min=1, ctx_max=1)
