@@ -25,7 +25,11 @@
 //   coalesced 16-byte stores.
 // Phase 3 (attention), per sequence of the group, on the tensor cores. K
 //   and V pages are gathered by TMA through the block table, two 64-slot
-//   pages per 128-key chunk, into a 3-slot ring.
+//   pages per 128-key chunk, into a 3-slot ring. A sequence of 16, 32 or 64
+//   padded rows whose chunks' scores fit the 512 TMEM columns keeps them
+//   resident: one S^T = K Q^T product per chunk, K read once, row maxima and
+//   sums reduced across lanes and lane quadrants, P formed from the same
+//   scores. Any other sequence takes two passes:
 //   Pass 1 finds every row's log-sum-exp from S = Q K^T with the rows on
 //   TMEM lanes, so each thread keeps its own row's running max and sum. A
 //   sequence of at most 64 rows is first repeated across the four lane
@@ -41,7 +45,8 @@
 //   accumulates both (O^T hi and lo in adjacent column ranges, summed when
 //   out is stored). The
 //   Flash-Verify two-view rule (paragraph 3 of the same page) decides
-//   visibility of fresh view keys.
+//   visibility of fresh view keys, read from a table the tile builds once
+//   (one 32-bit word per view slot and 32 rows).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
